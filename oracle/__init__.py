@@ -1,0 +1,178 @@
+"""fp64 CPU oracle for the DSA hot path -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never calls it and
+shares no code with it.
+
+``oracle.c`` holds the definitions (compiled to ``liboracle.so`` with gcc);
+this module marshals numpy arrays into it.  ``brute.py`` holds independent
+tiny-input brute-force versions used to pin ``oracle.c``.
+
+Every function follows the plain definition of its stage, as the pages state
+it ("DeepSeek V3.2 and the lightning indexer", section "How the lightning
+indexer works"; "DeepSeek-V3.2" atlas entry, "Design overview"):
+
+* indexer  I[t,s] = sum_j w[t,j] * ReLU(qhat[t,j] . khat[s])  for s <= p
+* top-k    the min(k, p+1) best scores, ties to the lower index, ascending
+* attention softmax over the selected latents, shared by all query heads
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (gcc, -O2, OpenMP, IEEE math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-Wall",
+               "-o", _LIB, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        i32 = ctypes.c_int
+        lib.oracle_e4m3_decode.restype = ctypes.c_double
+        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_bf16_decode.restype = ctypes.c_double
+        lib.oracle_bf16_decode.argtypes = [ctypes.c_uint16]
+        lib.oracle_indexer.restype = i32
+        lib.oracle_indexer.argtypes = [P, P, P, P, P, i64, i64, i32, i32, P, i64, P, i64]
+        lib.oracle_topk.restype = i32
+        lib.oracle_topk.argtypes = [P, i64, i64, i64, P, i64, i32, P]
+        lib.oracle_sparse_mla.restype = i32
+        lib.oracle_sparse_mla.argtypes = [P, P, P, i64, i64, i32, i32, i32, i32, ctypes.c_double,
+                                          P, i64, P, P]
+        lib.oracle_forward.restype = i32
+        lib.oracle_forward.argtypes = [P, P, P, P, P, P, P, i64, i64, i32, i32, i32, i32, i32, i32,
+                                       ctypes.c_double, P, i64, P, P, P]
+        lib.oracle_num_threads.restype = i32
+        lib.oracle_num_threads.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle inputs must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _rows(rows, n_q):
+    if rows is None:
+        return np.arange(n_q, dtype=np.int64)
+    return _c(rows, np.int64)
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def e4m3_decode(b: int) -> float:
+    return float(_load().oracle_e4m3_decode(int(b) & 0xFF))
+
+
+def bf16_decode(h: int) -> float:
+    return float(_load().oracle_bf16_decode(int(h) & 0xFFFF))
+
+
+def indexer(q8, q_scale, w, k8, k_scale, rows=None) -> np.ndarray:
+    """Indexer scores for one sequence.
+
+    q8: uint8 [n_q, H_I, d_I] (e4m3 bytes); q_scale, w: float32 [n_q, H_I];
+    k8: uint8 [n_k, d_I]; k_scale: float32 [n_k].  Returns float64
+    [len(rows), n_k], NaN where s > p (p = n_k - n_q + i).
+    """
+    q8 = _c(q8, np.uint8)
+    k8 = _c(k8, np.uint8)
+    n_q, H_I, d_I = q8.shape
+    n_k = k8.shape[0]
+    rows = _rows(rows, n_q)
+    out = np.full((len(rows), n_k), np.nan, dtype=np.float64)
+    rc = _load().oracle_indexer(_ptr(q8), _ptr(_c(q_scale, np.float32)), _ptr(_c(w, np.float32)),
+                                _ptr(k8), _ptr(_c(k_scale, np.float32)), n_q, n_k, H_I, d_I,
+                                _ptr(rows), len(rows), _ptr(out), n_k)
+    if rc != 0:
+        raise ValueError("oracle_indexer: bad arguments")
+    return out
+
+
+def topk(scores, n_q, k, rows=None) -> np.ndarray:
+    """Top-k for one sequence: scores float64 [len(rows), n_k] (candidates of
+    row r at 0..p_r).  Returns int32 [len(rows), k], ascending, -1 padded."""
+    scores = _c(scores, np.float64)
+    n_k = scores.shape[1]
+    rows = _rows(rows, n_q)
+    assert scores.shape[0] == len(rows)
+    idx = np.empty((len(rows), k), dtype=np.int32)
+    rc = _load().oracle_topk(_ptr(scores), n_k, n_q, n_k, _ptr(rows), len(rows), k, _ptr(idx))
+    if rc != 0:
+        raise ValueError("oracle_topk: bad arguments")
+    return idx
+
+
+def sparse_mla(q_bits, kv_bits, idx, n_k, scale, d_v=512, rows=None):
+    """Sparse MQA-mode attention for one sequence.
+
+    q_bits: uint16 [n_q, H, d_qk] (bf16 bit patterns); kv_bits: uint16
+    [n_k, d_qk]; idx: int32 [len(rows), k].  Returns (out float64
+    [len(rows), H, d_v], lse float64 [len(rows), H]).
+    """
+    q_bits = _c(q_bits, np.uint16)
+    kv_bits = _c(kv_bits, np.uint16)
+    idx = _c(idx, np.int32)
+    n_q, H, d_qk = q_bits.shape
+    assert kv_bits.shape == (n_k, d_qk)
+    rows = _rows(rows, n_q)
+    k = idx.shape[1]
+    out = np.empty((len(rows), H, d_v), dtype=np.float64)
+    lse = np.empty((len(rows), H), dtype=np.float64)
+    rc = _load().oracle_sparse_mla(_ptr(q_bits), _ptr(kv_bits), _ptr(idx), n_q, n_k, H, d_qk, d_v,
+                                   k, float(scale), _ptr(rows), len(rows), _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_sparse_mla: bad arguments")
+    return out, lse
+
+
+def forward(q8, q_scale, w, k8, k_scale, q_bits, kv_bits, k, scale, d_v=512, rows=None):
+    """indexer -> top-k -> sparse attention for the listed rows of one
+    sequence.  Returns (idx int32 [R, k], out float64 [R, H, d_v], lse [R, H])."""
+    q8 = _c(q8, np.uint8)
+    k8 = _c(k8, np.uint8)
+    q_bits = _c(q_bits, np.uint16)
+    kv_bits = _c(kv_bits, np.uint16)
+    n_q, H_I, d_I = q8.shape
+    n_k = k8.shape[0]
+    _, H, d_qk = q_bits.shape
+    rows = _rows(rows, n_q)
+    R = len(rows)
+    idx = np.empty((R, k), dtype=np.int32)
+    out = np.empty((R, H, d_v), dtype=np.float64)
+    lse = np.empty((R, H), dtype=np.float64)
+    rc = _load().oracle_forward(_ptr(q8), _ptr(_c(q_scale, np.float32)), _ptr(_c(w, np.float32)),
+                                _ptr(k8), _ptr(_c(k_scale, np.float32)), _ptr(q_bits),
+                                _ptr(kv_bits), n_q, n_k, H_I, d_I, H, d_qk, d_v, k, float(scale),
+                                _ptr(rows), R, _ptr(idx), _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_forward: bad arguments")
+    return idx, out, lse

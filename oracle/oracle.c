@@ -1,0 +1,321 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU oracle for the DeepSeek Sparse Attention
+ * (DSA) hot path: lightning-indexer scores -> per-query top-k -> sparse
+ * attention in the MQA mode of MLA.
+ *
+ * THIS IS TEST INFRASTRUCTURE.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg load it.  It shares no code, header, table or
+ * constant with the CUDA library, and the CUDA library never calls it.
+ *
+ * Everything is computed in double precision straight from the definitions,
+ * one query row at a time, with no blocking, fusion or reordering.  OpenMP
+ * only spreads independent query rows over host cores.
+ *
+ * Sources (the pages this follows):
+ *  - "DeepSeek V3.2 and the lightning indexer" (montana-research blog),
+ *    section "How the lightning indexer works": the indexer score between a
+ *    query and each earlier token is a weighted sum of ReLU-activated dot
+ *    products computed by a few indexer heads, in FP8; the top 2,048 entries
+ *    per query are kept and the main attention runs only over them; DSA runs on
+ *    the MQA mode of MLA, so one selected latent is shared by every query head
+ *    and the selection is made once per query position.
+ *  - "DeepSeek-V3.2" (atlas.lewiswon.me), "Design overview" and the
+ *    "Inference efficiency" row of the spec sheet: a few indexer heads score
+ *    every query against all earlier tokens with ReLU and per-head weights;
+ *    token-level top-k with k = 2048 per query; the main attention reads only
+ *    the chosen latents.
+ *  - "DeepSeek-V3.2 ... (introducing DSA)" (phantomic12 paper record): the FP8
+ *    ReLU indexer yields one scalar logit per (query, KV) pair; only the top-k
+ *    of those are attended.
+ *
+ * Readings where the pages are silent:
+ *  - causal: the query at absolute position p may use keys 0..p (self
+ *    included); in a sequence with n_k keys and n_q queries the local query i
+ *    sits at p = (n_k - n_q) + i;
+ *  - indexer: I[t,s] = sum_j w[t,j] * max(0, qhat[t,j,:] . khat[s,:]) with
+ *    qhat = e4m3(q8) * q_scale[t,j] and khat = e4m3(k8) * k_scale[s];
+ *  - top-k: the min(k, p+1) largest scores, ties to the lower index, -0 equal
+ *    to +0, emitted in ascending index order and padded with -1;
+ *  - attention: o[t,h] = sum_s softmax_s(scale * q[t,h,:] . c[s,:]) * c[s,0:d_v]
+ *    over the selected set, lse = log sum_s exp(scale * q . c).
+ *
+ * Parity pins: tests/test_oracle_pins.py checks every function here against
+ * brute force, closed forms, invariants and library routines.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---------------------------------------------------------------------- */
+/* Number formats.                                                         */
+/* ---------------------------------------------------------------------- */
+
+/* FP8 E4M3 ("fn" variant: no infinities, 0x7F/0xFF are NaN): 1 sign bit,
+ * 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0 encodes the
+ * subnormals m * 2^-9.  Decoded from the bit fields, not from a table copied
+ * from anywhere. */
+double oracle_e4m3_decode(uint8_t b) {
+  int sign = (b >> 7) & 1;
+  int e = (b >> 3) & 15;
+  int m = b & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0)
+    v = ldexp((double)m, -9); /* m/8 * 2^(1-7) */
+  else
+    v = ldexp(1.0 + (double)m / 8.0, e - 7);
+  return sign ? -v : v;
+}
+
+/* bfloat16 is the top half of an IEEE binary32. */
+double oracle_bf16_decode(uint16_t h) {
+  uint32_t u = ((uint32_t)h) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Lightning indexer.                                                       */
+/* ---------------------------------------------------------------------- */
+
+/* Score of query row i against key s (blog, "How the lightning indexer
+ * works": weighted sum over indexer heads of ReLU(query-head . key)). */
+static double indexer_score(const uint8_t* q8, const float* q_scale, const float* w,
+                            const uint8_t* k8, const float* k_scale, int64_t i, int64_t s,
+                            int H_I, int d_I) {
+  double total = 0.0;
+  for (int j = 0; j < H_I; ++j) {
+    const uint8_t* qrow = q8 + ((int64_t)i * H_I + j) * d_I;
+    const uint8_t* krow = k8 + (int64_t)s * d_I;
+    double qs = (double)q_scale[(int64_t)i * H_I + j];
+    double ks = (double)k_scale[s];
+    double dot = 0.0;
+    for (int d = 0; d < d_I; ++d)
+      dot += (oracle_e4m3_decode(qrow[d]) * qs) * (oracle_e4m3_decode(krow[d]) * ks);
+    double relu = dot > 0.0 ? dot : 0.0;
+    total += (double)w[(int64_t)i * H_I + j] * relu;
+  }
+  return total;
+}
+
+/* For each listed local query row i (rows == NULL means rows 0..n_rows-1),
+ * writes I[i, s] for s = 0..p_i into out[r * ld_out + s], p_i = n_k - n_q + i.
+ * Entries s > p_i are left untouched.  Returns 0, or -1 on bad arguments. */
+int oracle_indexer(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8,
+                   const float* k_scale, int64_t n_q, int64_t n_k, int H_I, int d_I,
+                   const int64_t* rows, int64_t n_rows, double* out, int64_t ld_out) {
+  if (n_q < 0 || n_k < n_q || H_I <= 0 || d_I <= 0 || ld_out < n_k) return -1;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    int64_t i = rows ? rows[r] : r;
+    if (i < 0 || i >= n_q) {
+      bad = 1;
+      continue;
+    }
+    int64_t p = n_k - n_q + i;
+    for (int64_t s = 0; s <= p; ++s)
+      out[r * ld_out + s] = indexer_score(q8, q_scale, w, k8, k_scale, i, s, H_I, d_I);
+  }
+  return bad ? -1 : 0;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Top-k selection.                                                         */
+/* ---------------------------------------------------------------------- */
+
+typedef struct {
+  double v;
+  int64_t s;
+} scored_t;
+
+/* Descending score, then ascending index.  -0.0 == +0.0 under IEEE compare,
+ * so the two zeros are one value here. */
+static int by_score_desc_index_asc(const void* a, const void* b) {
+  const scored_t* x = (const scored_t*)a;
+  const scored_t* y = (const scored_t*)b;
+  if (x->v > y->v) return -1;
+  if (x->v < y->v) return 1;
+  return (x->s > y->s) - (x->s < y->s);
+}
+
+static int by_index_asc(const void* a, const void* b) {
+  int32_t x = *(const int32_t*)a, y = *(const int32_t*)b;
+  return (x > y) - (x < y);
+}
+
+/* Selects, for one row of n = p + 1 candidate scores, the min(k, n) largest
+ * by a full sort (blog, "How the lightning indexer works": a fixed number of
+ * best-scoring entries is kept per query), writes them in ascending index order to idx[0..k) and pads with -1.
+ * scratch holds at least n entries. */
+static void topk_row(const double* scores, int64_t n, int k, scored_t* scratch, int32_t* idx) {
+  for (int64_t s = 0; s < n; ++s) {
+    double v = scores[s];
+    if (v == 0.0) v = 0.0; /* -0 -> +0 */
+    scratch[s].v = v;
+    scratch[s].s = s;
+  }
+  qsort(scratch, (size_t)n, sizeof(scored_t), by_score_desc_index_asc);
+  int64_t m = n < k ? n : k;
+  for (int64_t r = 0; r < m; ++r) idx[r] = (int32_t)scratch[r].s;
+  qsort(idx, (size_t)m, sizeof(int32_t), by_index_asc);
+  for (int64_t r = m; r < k; ++r) idx[r] = -1;
+}
+
+/* scores: n_rows rows of stride ld; row r holds its candidates at 0..p_r,
+ * p_r = n_k - n_q + rows[r].  idx_out: n_rows x k int32. */
+int oracle_topk(const double* scores, int64_t ld, int64_t n_q, int64_t n_k, const int64_t* rows,
+                int64_t n_rows, int k, int32_t* idx_out) {
+  if (k <= 0 || n_k < n_q || ld < n_k) return -1;
+  int bad = 0;
+#pragma omp parallel
+  {
+    scored_t* scratch = (scored_t*)malloc(sizeof(scored_t) * (size_t)(n_k > 0 ? n_k : 1));
+#pragma omp for schedule(dynamic, 4)
+    for (int64_t r = 0; r < n_rows; ++r) {
+      int64_t i = rows ? rows[r] : r;
+      if (i < 0 || i >= n_q || !scratch) {
+        bad = 1;
+        continue;
+      }
+      int64_t p = n_k - n_q + i;
+      topk_row(scores + r * ld, p + 1, k, scratch, idx_out + r * (int64_t)k);
+    }
+    free(scratch);
+  }
+  return bad ? -1 : 0;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Sparse attention, MQA mode of MLA.                                       */
+/* ---------------------------------------------------------------------- */
+
+/* One query row, all heads, over the selected set sel[0..n_sel).
+ * Latent c[s] has d_qk dims; its first d_v dims are the value.  (blog, "How
+ * the lightning indexer works": each latent is shared by all query heads.) */
+static void attend_row(const uint16_t* q, const uint16_t* kv, const int32_t* sel, int64_t n_sel,
+                       int64_t i, int H, int d_qk, int d_v, double scale, double* o, double* lse,
+                       double* x) {
+  for (int h = 0; h < H; ++h) {
+    const uint16_t* qh = q + ((int64_t)i * H + h) * d_qk;
+    double m = -INFINITY;
+    for (int64_t r = 0; r < n_sel; ++r) {
+      const uint16_t* c = kv + (int64_t)sel[r] * d_qk;
+      double dot = 0.0;
+      for (int d = 0; d < d_qk; ++d) dot += oracle_bf16_decode(qh[d]) * oracle_bf16_decode(c[d]);
+      x[r] = scale * dot;
+      if (x[r] > m) m = x[r];
+    }
+    double* oh = o + (int64_t)h * d_v;
+    for (int d = 0; d < d_v; ++d) oh[d] = 0.0;
+    double z = 0.0;
+    for (int64_t r = 0; r < n_sel; ++r) {
+      double e = exp(x[r] - m);
+      z += e;
+      const uint16_t* c = kv + (int64_t)sel[r] * d_qk;
+      for (int d = 0; d < d_v; ++d) oh[d] += e * oracle_bf16_decode(c[d]);
+    }
+    if (n_sel == 0) {
+      lse[h] = -INFINITY;
+      continue;
+    }
+    for (int d = 0; d < d_v; ++d) oh[d] /= z;
+    lse[h] = m + log(z);
+  }
+}
+
+/* Keeps the entries of an index row that name a key the query may use
+ * (0 <= s <= p), in row order. */
+static int64_t valid_entries(const int32_t* idx_row, int k, int64_t p, int32_t* sel) {
+  int64_t n = 0;
+  for (int r = 0; r < k; ++r)
+    if (idx_row[r] >= 0 && idx_row[r] <= p) sel[n++] = idx_row[r];
+  return n;
+}
+
+/* q: n_q x H x d_qk bf16; kv: n_k x d_qk bf16; idx: n_rows x k (row r belongs
+ * to local query rows[r]).  out: n_rows x H x d_v; lse: n_rows x H. */
+int oracle_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int64_t n_q,
+                      int64_t n_k, int H, int d_qk, int d_v, int k, double scale,
+                      const int64_t* rows, int64_t n_rows, double* out, double* lse) {
+  if (k <= 0 || n_k < n_q || d_v > d_qk || H <= 0) return -1;
+  int bad = 0;
+#pragma omp parallel
+  {
+    int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+    double* x = (double*)malloc(sizeof(double) * (size_t)k);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; ++r) {
+      int64_t i = rows ? rows[r] : r;
+      if (i < 0 || i >= n_q || !sel || !x) {
+        bad = 1;
+        continue;
+      }
+      int64_t p = n_k - n_q + i;
+      int64_t n_sel = valid_entries(idx + r * (int64_t)k, k, p, sel);
+      attend_row(q, kv, sel, n_sel, i, H, d_qk, d_v, scale, out + r * (int64_t)H * d_v,
+                 lse + r * (int64_t)H, x);
+    }
+    free(sel);
+    free(x);
+  }
+  return bad ? -1 : 0;
+}
+
+/* ---------------------------------------------------------------------- */
+/* The whole path for selected query rows.                                  */
+/* ---------------------------------------------------------------------- */
+
+/* indexer -> top-k -> sparse attention, one query row at a time.  idx_out
+ * (n_rows x k), out (n_rows x H x d_v) and lse (n_rows x H) receive the
+ * results; idx_out may be NULL. */
+int oracle_forward(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8,
+                   const float* k_scale, const uint16_t* q, const uint16_t* kv, int64_t n_q,
+                   int64_t n_k, int H_I, int d_I, int H, int d_qk, int d_v, int k, double scale,
+                   const int64_t* rows, int64_t n_rows, int32_t* idx_out, double* out,
+                   double* lse) {
+  if (k <= 0 || n_k < n_q || d_v > d_qk || H <= 0 || H_I <= 0 || d_I <= 0) return -1;
+  int bad = 0;
+#pragma omp parallel
+  {
+    double* scores = (double*)malloc(sizeof(double) * (size_t)(n_k > 0 ? n_k : 1));
+    scored_t* scratch = (scored_t*)malloc(sizeof(scored_t) * (size_t)(n_k > 0 ? n_k : 1));
+    int32_t* idx = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+    int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+    double* x = (double*)malloc(sizeof(double) * (size_t)k);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; ++r) {
+      int64_t i = rows ? rows[r] : r;
+      if (i < 0 || i >= n_q || !scores || !scratch || !idx || !sel || !x) {
+        bad = 1;
+        continue;
+      }
+      int64_t p = n_k - n_q + i;
+      for (int64_t s = 0; s <= p; ++s)
+        scores[s] = indexer_score(q8, q_scale, w, k8, k_scale, i, s, H_I, d_I);
+      topk_row(scores, p + 1, k, scratch, idx);
+      if (idx_out) memcpy(idx_out + r * (int64_t)k, idx, sizeof(int32_t) * (size_t)k);
+      int64_t n_sel = valid_entries(idx, k, p, sel);
+      attend_row(q, kv, sel, n_sel, i, H, d_qk, d_v, scale, out + r * (int64_t)H * d_v,
+                 lse + r * (int64_t)H, x);
+    }
+    free(scores);
+    free(scratch);
+    free(idx);
+    free(sel);
+    free(x);
+  }
+  return bad ? -1 : 0;
+}
+
+/* Threads OpenMP will use (reported beside the CPU baseline). */
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  extern int omp_get_max_threads(void);
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}

@@ -1,0 +1,322 @@
+"""Pins of the fp64 oracle to things other than itself (CPU only).
+
+Each test checks the oracle against a closed form, an invariant, brute force
+on tiny inputs, or a library routine, so that a dropped term, a wrong sign or
+index, or a transposed operand in ``oracle/oracle.c`` fails at least one.
+
+Pages: "DeepSeek V3.2 and the lightning indexer", section "How the lightning
+indexer works" (indexer = weighted sum of ReLU'd dot products per indexer
+head, FP8; fixed top-k per query; MQA mode of MLA); "DeepSeek-V3.2" atlas
+entry, "Design overview" (score against every preceding token, k = 2048).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import brute
+from sparse_attention_08_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+def _e4m3_to_f64(b):
+    return torch.from_numpy(np.ascontiguousarray(b)).view(torch.float8_e4m3fn).to(
+        torch.float64).numpy()
+
+
+def _bf16_to_f64(t):
+    return t.to(torch.float64).numpy()
+
+
+def _bits(t_bf16):
+    return _np(t_bf16.contiguous().view(torch.int16)).view(np.uint16)
+
+
+# --------------------------------------------------------------------------
+# Number formats: against torch's own conversions (library routines).
+# --------------------------------------------------------------------------
+
+def test_e4m3_decode_matches_torch_all_codes():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = _e4m3_to_f64(codes)
+    for b in range(256):
+        v = oracle.e4m3_decode(b)
+        if math.isnan(ref[b]):
+            assert math.isnan(v), hex(b)
+        else:
+            assert v == ref[b], (hex(b), v, ref[b])
+    # spot values fixed by the format: 1.0, max normal 448, min subnormal 2^-9
+    assert oracle.e4m3_decode(0x38) == 1.0
+    assert oracle.e4m3_decode(0x7E) == 448.0
+    assert oracle.e4m3_decode(0x01) == 2.0 ** -9
+    assert oracle.e4m3_decode(0xB8) == -1.0
+
+
+def test_bf16_decode_matches_torch():
+    g = torch.Generator().manual_seed(1)
+    x = (torch.randn(4096, generator=g) * 100).to(torch.bfloat16)
+    bits = _bits(x)
+    ref = x.to(torch.float64).numpy()
+    got = np.array([oracle.bf16_decode(int(b)) for b in bits])
+    assert np.array_equal(got, ref)
+
+
+# --------------------------------------------------------------------------
+# Indexer.
+# --------------------------------------------------------------------------
+
+def test_indexer_integer_inputs_exact_vs_int_brute_force():
+    # Integer-valued e4m3 codes with unit scales make every score an exact
+    # integer; exact Python-int arithmetic must be matched to the last bit.
+    wl = W.make_small(H_I=3, d_I=16, H=2, L=40, k=8, integer=True, seed=11)
+    q8, k8 = _np(wl.q8), _np(wl.k8)
+    q_int = np.vectorize(brute.int_of_e4m3_code, otypes=[object])(q8)
+    k_int = np.vectorize(brute.int_of_e4m3_code, otypes=[object])(k8)
+    w_int = _np(wl.w).astype(np.int64).astype(object)
+    exact = brute.indexer_int(q_int, w_int, k_int)
+    got = oracle.indexer(q8, _np(wl.q_scale), _np(wl.w), k8, _np(wl.k_scale))
+    n = wl.T_q
+    for i in range(n):
+        for s in range(n):
+            if s <= i:
+                assert got[i, s] == float(exact[i, s]), (i, s)
+            else:
+                assert math.isnan(got[i, s])
+
+
+def test_indexer_fold_identity_real_valued():
+    # Dequantise-then-dot (oracle) equals the folded form
+    # k_scale[s] * sum_j (w*q_scale)[t,j] * ReLU(q8[t,j] . k8[s]) built here from
+    # torch's e4m3 decode: positive scales pass through the ReLU.
+    wl = W.make_small(H_I=8, d_I=32, H=2, L=50, k=8, seed=12)
+    q8, k8 = _np(wl.q8), _np(wl.k8)
+    qd = _e4m3_to_f64(q8)
+    kd = _e4m3_to_f64(k8)
+    raw = np.einsum("tjd,sd->tjs", qd, kd)
+    wq = _np(wl.w).astype(np.float64) * _np(wl.q_scale).astype(np.float64)
+    folded = np.einsum("tj,tjs->ts", wq, np.maximum(raw, 0.0)) * _np(wl.k_scale).astype(
+        np.float64)[None, :]
+    got = oracle.indexer(q8, _np(wl.q_scale), _np(wl.w), k8, _np(wl.k_scale))
+    mask = np.tril(np.ones((wl.T_q, wl.T_k), dtype=bool))
+    denom = np.einsum("tj,tjs->ts", np.abs(wq), np.maximum(raw, 0.0)) * _np(wl.k_scale)[None, :]
+    err = np.abs(got[mask] - folded[mask])
+    assert np.all(err <= 1e-12 * denom[mask] + 1e-300)
+
+
+def test_indexer_invariants():
+    wl = W.make_small(H_I=4, d_I=16, H=2, L=30, k=8, seed=13)
+    q8, k8 = _np(wl.q8), _np(wl.k8).copy()
+    qs, w, ks = _np(wl.q_scale), _np(wl.w), _np(wl.k_scale).copy()
+    base = oracle.indexer(q8, qs, w, k8, ks)
+    mask = np.tril(np.ones(base.shape, dtype=bool))
+    # doubling a key's scale doubles its scores exactly (power-of-two scaling)
+    ks2 = ks.copy()
+    ks2[7] *= 2
+    dbl = oracle.indexer(q8, qs, w, k8, ks2)
+    assert np.array_equal(dbl[7:, 7], 2 * base[7:, 7])
+    assert np.array_equal(np.delete(dbl, 7, axis=1)[np.delete(mask, 7, axis=1)],
+                          np.delete(base, 7, axis=1)[np.delete(mask, 7, axis=1)])
+    # a zero key scores zero against every query
+    k8z = k8.copy()
+    k8z[5] = 0
+    z = oracle.indexer(q8, qs, w, k8z, ks)
+    assert np.all(z[5:, 5] == 0.0)
+    # one-hot head weights isolate one ReLU term, which is never negative,
+    # and the terms add up to the score
+    acc = np.zeros_like(base)
+    for j in range(4):
+        wj = np.zeros_like(w)
+        wj[:, j] = w[:, j]
+        one = np.zeros_like(w)
+        one[:, j] = 1.0
+        term = oracle.indexer(q8, qs, one, k8, ks)
+        assert np.all(term[mask] >= 0.0)
+        acc += oracle.indexer(q8, qs, wj, k8, ks)
+    assert np.allclose(acc[mask], base[mask], rtol=1e-13, atol=1e-300)
+    # non-negative weights give non-negative scores
+    pos = oracle.indexer(q8, qs, np.abs(w), k8, ks)
+    assert np.all(pos[mask] >= 0.0)
+    # a negative weight flips the sign of that head's (non-negative) term
+    neg = oracle.indexer(q8, qs, -np.abs(w), k8, ks)
+    assert np.all(neg[mask] <= 0.0)
+    assert np.array_equal(neg[mask], -pos[mask])
+
+
+# --------------------------------------------------------------------------
+# Top-k.
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_topk_matches_full_sort_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    n_q, n_k, k = 37, 60, 9
+    # integer scores -> many exact ties; include signed zeros
+    scores = rng.integers(-3, 4, size=(n_q, n_k)).astype(np.float64)
+    scores[rng.random(scores.shape) < 0.1] = -0.0
+    got = oracle.topk(scores, n_q, k)
+    for i in range(n_q):
+        p = n_k - n_q + i
+        assert list(got[i]) == brute.topk_sorted(scores[i], p, k), i
+
+
+def test_topk_counts_ties_and_zero_signs():
+    n_q = n_k = 20
+    k = 6
+    ties = np.zeros((n_q, n_k))
+    got = oracle.topk(ties, n_q, k)
+    for i in range(n_q):
+        m = min(k, i + 1)                       # O(Lk): min(k, p+1) entries per row
+        assert list(got[i][:m]) == list(range(m))
+        assert np.all(got[i][m:] == -1)
+    # -0.0 and +0.0 are the same value: the lower index wins
+    row = np.full((1, 4), -1.0)
+    row[0, 1] = -0.0
+    row[0, 3] = 0.0
+    assert list(oracle.topk(row, 1, 1, rows=None)[0]) == [1]
+    row[0, 1], row[0, 3] = 0.0, -0.0
+    assert list(oracle.topk(row, 1, 1)[0]) == [1]
+
+
+def test_topk_selects_largest_real_scores():
+    rng = np.random.default_rng(5)
+    scores = rng.standard_normal((1, 500))
+    got = oracle.topk(scores, 1, 50)[0]
+    ref = np.sort(np.argsort(-scores[0], kind="stable")[:50])
+    assert np.array_equal(got, ref)
+
+
+# --------------------------------------------------------------------------
+# Attention.
+# --------------------------------------------------------------------------
+
+def _sdpa_dense(q_bf16, kv_bf16, n_k, scale, d_v):
+    """Dense causal MQA attention in fp64 by torch's SDPA (library routine)."""
+    q = q_bf16.to(torch.float64).permute(1, 0, 2)[None]          # [1, H, n_q, d]
+    k = kv_bf16.to(torch.float64)[None, None]                    # [1, 1, n_k, d]
+    v = kv_bf16[:, :d_v].to(torch.float64)[None, None]
+    n_q = q.shape[2]
+    H = q.shape[1]
+    pos = torch.arange(n_q)[:, None] + (n_k - n_q)
+    mask = torch.arange(n_k)[None, :] <= pos
+    out = torch.nn.functional.scaled_dot_product_attention(
+        q, k.expand(1, H, n_k, -1), v.expand(1, H, n_k, -1), attn_mask=mask, scale=scale)
+    return out[0].permute(1, 0, 2).numpy()                       # [n_q, H, d_v]
+
+
+def test_attention_dense_limit_matches_sdpa():
+    # With p+1 <= k every causal key is selected: sparse == dense causal MQA.
+    wl = W.make_small(H_I=4, d_I=16, H=4, L=48, k=64, seed=21)
+    scores = oracle.indexer(_np(wl.q8), _np(wl.q_scale), _np(wl.w), _np(wl.k8), _np(wl.k_scale))
+    idx = oracle.topk(np.nan_to_num(scores, nan=0.0), wl.T_q, wl.k)
+    out, lse = oracle.sparse_mla(_bits(wl.q), _bits(wl.kv), idx, wl.T_k, wl.scale, d_v=512)
+    ref = _sdpa_dense(wl.q, wl.kv, wl.T_k, wl.scale, 512)
+    assert np.max(np.abs(out - ref)) < 1e-12
+
+
+def test_attention_k_equals_L_is_dense_exactly():
+    # k = L: the selection is every causal key, in ascending order, so the
+    # result is bitwise that of attention over the explicit causal index list.
+    wl = W.make_small(H_I=4, d_I=16, H=3, L=40, k=40, seed=22)
+    idx, out, lse = oracle.forward(_np(wl.q8), _np(wl.q_scale), _np(wl.w), _np(wl.k8),
+                                   _np(wl.k_scale), _bits(wl.q), _bits(wl.kv), wl.k, wl.scale)
+    dense_idx = np.full((wl.T_q, wl.k), -1, dtype=np.int32)
+    for i in range(wl.T_q):
+        dense_idx[i, : i + 1] = np.arange(i + 1)
+    assert np.array_equal(idx, dense_idx)
+    out2, lse2 = oracle.sparse_mla(_bits(wl.q), _bits(wl.kv), dense_idx, wl.T_k, wl.scale)
+    assert np.array_equal(out, out2) and np.array_equal(lse, lse2)
+    ref = _sdpa_dense(wl.q, wl.kv, wl.T_k, wl.scale, 512)
+    assert np.max(np.abs(out - ref)) < 1e-12
+
+
+def test_attention_single_key_and_zero_query():
+    wl = W.make_small(H_I=4, d_I=16, H=2, L=30, k=4, seed=23)
+    idx = np.full((wl.T_q, 4), -1, dtype=np.int32)
+    for i in range(wl.T_q):
+        idx[i, 0] = i // 2
+    out, _ = oracle.sparse_mla(_bits(wl.q), _bits(wl.kv), idx, wl.T_k, wl.scale)
+    kvd = _bf16_to_f64(wl.kv)
+    for i in range(wl.T_q):
+        assert np.array_equal(out[i, 0], kvd[i // 2, :512])
+        assert np.array_equal(out[i, 1], kvd[i // 2, :512])
+    # q = 0: uniform softmax, output = mean of the selected values
+    qz = torch.zeros_like(wl.q)
+    idx2 = np.full((wl.T_q, 4), -1, dtype=np.int32)
+    for i in range(wl.T_q):
+        sel = sorted({0, i // 2, i})
+        idx2[i, : len(sel)] = sel
+    out0, lse0 = oracle.sparse_mla(_bits(qz), _bits(wl.kv), idx2, wl.T_k, wl.scale)
+    for i in range(wl.T_q):
+        sel = [s for s in idx2[i] if s >= 0]
+        assert np.allclose(out0[i, 0], kvd[sel, :512].mean(axis=0), rtol=0, atol=1e-15)
+        assert abs(lse0[i, 0] - math.log(len(sel))) < 1e-15
+
+
+def test_attention_matches_explicit_loops_and_skips_invalid():
+    wl = W.make_small(H_I=4, d_I=16, H=2, L=25, k=7, seed=24, q_div=2.0)
+    rng = np.random.default_rng(3)
+    idx = np.full((wl.T_q, 7), -1, dtype=np.int32)
+    for i in range(wl.T_q):
+        m = min(7, i + 1)
+        idx[i, :m] = np.sort(rng.choice(i + 1, size=m, replace=False))
+    idx[3, 1] = 24          # beyond p = 3: skipped
+    out, lse = oracle.sparse_mla(_bits(wl.q), _bits(wl.kv), idx, wl.T_k, wl.scale)
+    qd, kvd = _bf16_to_f64(wl.q), _bf16_to_f64(wl.kv)
+    for i in range(wl.T_q):
+        sel = [int(s) for s in idx[i] if 0 <= s <= i]
+        ro, rl = brute.attention_loops(qd[i], kvd, sel, wl.scale, 512)
+        assert np.max(np.abs(out[i] - ro)) < 1e-13
+        assert np.max(np.abs(lse[i] - rl)) < 1e-13
+
+
+def test_forward_is_the_composition():
+    wl = W.make_small(H_I=4, d_I=16, H=2, lens=[30, 45], lens_q=[30, 20], k=8, seed=25)
+    # second sequence is a chunk: 20 queries at positions 25..44
+    b = 1
+    q0, q1 = int(wl.cu_q[b]), int(wl.cu_q[b + 1])
+    k0, k1 = int(wl.cu_k[b]), int(wl.cu_k[b + 1])
+    args = [_np(wl.q8[q0:q1]), _np(wl.q_scale[q0:q1]), _np(wl.w[q0:q1]), _np(wl.k8[k0:k1]),
+            _np(wl.k_scale[k0:k1])]
+    rows = np.array([0, 3, 19], dtype=np.int64)
+    idx, out, lse = oracle.forward(*args, _bits(wl.q[q0:q1]), _bits(wl.kv[k0:k1]), wl.k,
+                                   wl.scale, rows=rows)
+    sc = oracle.indexer(*args, rows=rows)
+    assert np.all(np.isnan(sc[0, 26:])) and not np.any(np.isnan(sc[0, :26]))
+    idx2 = oracle.topk(np.nan_to_num(sc, nan=0.0), q1 - q0, wl.k, rows=rows)
+    out2, lse2 = oracle.sparse_mla(_bits(wl.q[q0:q1]), _bits(wl.kv[k0:k1]), idx2, k1 - k0,
+                                   wl.scale, rows=rows)
+    assert np.array_equal(idx, idx2)
+    assert np.array_equal(out, out2) and np.array_equal(lse, lse2)
+
+
+# --------------------------------------------------------------------------
+# Golden fixtures from the pages.
+# --------------------------------------------------------------------------
+
+def test_golden_sparse_budget():
+    with open(os.path.join(GOLDEN, "sparse_budget.json")) as f:
+        g = json.load(f)
+    # "488x" at a 1M-token context with k = 2048: full L*L versus L*k work.
+    L, k = g["reduction"]["L"], g["reduction"]["k"]
+    assert round((L * L) / (L * k)) == g["reduction"]["ratio_rounded"]
+    # every row keeps min(k, p+1) entries: count them with the oracle on a
+    # small case and compare with the closed form stored beside it
+    c = g["row_counts"]
+    wl = W.make_small(H_I=2, d_I=16, H=1, L=c["L"], k=c["k"], seed=31)
+    sc = oracle.indexer(_np(wl.q8), _np(wl.q_scale), _np(wl.w), _np(wl.k8), _np(wl.k_scale))
+    idx = oracle.topk(np.nan_to_num(sc, nan=0.0), wl.T_q, wl.k)
+    assert int((idx >= 0).sum()) == c["attended_pairs"]
+    # closed forms for the headline shapes
+    for row in g["configs"]:
+        L, k = row["L"], row["k"]
+        assert k * (k + 1) // 2 + (L - k) * k == row["attended_pairs"]
+        assert L * (L + 1) // 2 == row["causal_pairs"]
