@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of the DSA hot path: lightning indexer (FP8) -> top-2048 ->
+sparse MQA-mode MLA attention, on synthetic data shaped like the headline
+workload (one 32768-token prefill, H_I=64, d_I=128, H=128, 576-d latents).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the whole path over one batch (one sequence per GPU).
+Prints ONE JSON line on rank 0.  With --gpus N > 1 it runs under torchrun,
+one rank per GPU; every rank runs its own sequence (data-parallel, no
+collective on the data path) and the step time is the maximum over ranks.
+``--impl reference`` times the CPU oracle (oracle/, fp64, host cores) on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "DSA query-tokens/s (indexer+top-2048+sparse MLA) at L=32K; % roofline"
+UNIT = "query-tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+KERNEL_FILES = {
+    "indexer_kernel": "sparse_attention_08_b200/csrc/indexer.cu",
+    "topk_kernel": "sparse_attention_08_b200/csrc/topk.cu",
+    "sparse_mla_kernel": "sparse_attention_08_b200/csrc/sparse_mla.cu",
+}
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def source_sha(kernel):
+    with open(os.path.join(ROOT, KERNEL_FILES[kernel]), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(kernel, workload):
+    """Per-launch DRAM bytes from profiles/traffic.txt, if the capture was taken
+    on the current source of the kernel (null otherwise)."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    for line in open(p):
+        parts = line.split()
+        if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and \
+                parts[1] == workload and parts[3] == source_sha(kernel):
+            return float(parts[2])
+    return None
+
+
+def counts(wl):
+    """Algorithmic work of one pass over the workload."""
+    causal, attended = 0, 0
+    for nq, nk in zip(wl.lens_q, wl.lens_k):
+        causal += nq * (nk - nq) + nq * (nq + 1) // 2
+        for i in range(nq):
+            attended += min(wl.k, nk - nq + i + 1)
+    H_I, d_I = wl.q8.shape[1], wl.q8.shape[2]
+    H = wl.q.shape[1]
+    return {
+        "causal_pairs": causal,
+        "attended_pairs": attended,
+        # FP8 products of the indexer contraction (2 flops per MAC)
+        "indexer_flops": 2 * H_I * d_I * causal,
+        # QK^T over 576 dims + PV over 512 dims for every head and attended pair
+        "attention_flops": attended * H * (2 * 576 + 2 * 512),
+        # top-k: read every causal score once, write k indices per query
+        "topk_bytes": 4 * causal + 4 * wl.k * sum(wl.lens_q),
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            self.path = f"/tmp/dsa_clocks_{os.getpid()}.csv"
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu)], stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[3]) if v.lower() == "active"})
+        pmax = max(r[2] for r in rows)
+        loaded = [r for r in rows if r[2] >= 0.5 * pmax] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows), "power_w_max": pmax}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(wl, n_rows, seed):
+    """Runs the oracle on n_rows query rows drawn uniformly over positions (all
+    host cores, one OpenMP region); returns (elapsed seconds, description)."""
+    import oracle
+    from tests import dsa_cases as C
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(wl.T_q, size=n_rows, replace=False)).astype(np.int64)
+    n_k = wl.lens_k[0]
+    k8, ks, kvb = C.np_(wl.k8[:n_k]), C.np_(wl.k_scale[:n_k]), C.bits(wl.kv[:n_k])
+    rt = torch.as_tensor(rows, device=wl.q8.device)
+    q8, qs, w = C.np_(wl.q8[rt]), C.np_(wl.q_scale[rt]), C.np_(wl.w[rt])
+    qb = C.bits(wl.q[rt])
+    pos = rows + (n_k - wl.T_q)
+    t0 = time.perf_counter()
+    oracle.forward_at(q8, qs, w, k8, ks, qb, kvb, pos, wl.k, wl.scale)
+    dt = time.perf_counter() - t0
+    return dt, f"{n_rows} query rows drawn uniformly over positions 0..{wl.T_q - 1}"
+
+
+def oracle_threads():
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import sparse_attention_08_b200 as dsa
+    from sparse_attention_08_b200 import workloads as W
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dsa.load()
+    cfg = W.CONFIGS[args.config]
+    seed = W.seed_of(args.config) + 1000 * rank
+    wl = W.make_prefill(args.config, device="cuda", seed=seed)
+    H_I, d_I, H = wl.q8.shape[1], wl.q8.shape[2], wl.q.shape[1]
+    ld = (wl.max_len_k + 3) // 4 * 4
+    logits = torch.empty((wl.T_q, ld), dtype=torch.float32, device="cuda")
+    idx = torch.empty((wl.T_q, wl.k), dtype=torch.int32, device="cuda")
+    out = torch.empty((wl.T_q, H, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((wl.T_q, H), dtype=torch.float32, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        dsa.dsa_indexer_logits(wl.q8, wl.q_scale, wl.w, wl.k8, wl.k_scale, wl.cu_q, wl.cu_k, wl.B,
+                               wl.max_len_q, wl.max_len_k, logits, ld, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        dsa.dsa_topk(logits, wl.cu_q, wl.cu_k, wl.B, wl.max_len_q, wl.max_len_k, wl.k, idx,
+                     ld_logits=ld, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        dsa.dsa_sparse_mla_fwd(wl.q, wl.kv, idx, wl.cu_q, wl.cu_k, wl.B, wl.max_len_q,
+                               wl.max_len_k, wl.scale, out, lse, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    if dsa.dsa_get_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier(device_ids=[local])
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(args.steps):
+        flush.fill_(float(i))           # evicts L2 between steps (outside the events)
+        step(evs[i])
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    if dsa.dsa_get_device_error() != 0:
+        raise RuntimeError("device error during the timed region")
+    st = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)]
+                   for i in range(args.steps)])             # ms per stage per step
+    step_ms = float(st.sum(axis=1).mean())
+    stage_ms = st.mean(axis=0)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([step_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms = float(t.item())
+    value = world * wl.T_q / (step_ms / 1e3)
+
+    # ---- roofline of the dominant kernel and of the whole step
+    peaks = measured_peaks()
+    c = counts(wl)
+    fp8_peak = 2.0 * peaks["bf16_tflops_sustained"]     # nominal fp8:bf16 ratio 2
+    bf16_peak = peaks["bf16_tflops_sustained"]
+    names = ("indexer_kernel", "topk_kernel", "sparse_mla_kernel")
+    per = {
+        "indexer_kernel": ("tensor", c["indexer_flops"] / (stage_ms[0] / 1e3) / 1e12, fp8_peak,
+                           "TFLOP/s"),
+        "topk_kernel": ("hbm", c["topk_bytes"] / (stage_ms[1] / 1e3) / 1e9, peaks["hbm_gbs"],
+                        "GB/s"),
+        "sparse_mla_kernel": ("tensor", c["attention_flops"] / (stage_ms[2] / 1e3) / 1e12,
+                              bf16_peak, "TFLOP/s"),
+    }
+    dom = names[int(np.argmax(stage_ms))]
+    bound, ach, peak, unit = per[dom]
+    workload_name = f"{cfg.name}"
+    roofline = {"kernel": dom, "bound": bound, "achieved": round(ach, 2), "peak": peak,
+                "unit": unit, "frac": round(ach / peak, 4),
+                "traffic": ncu_traffic(dom, workload_name),
+                "peak_source": f"{peaks['source']} (sustained bf16" +
+                               (", x2 for fp8)" if dom == "indexer_kernel" else ")")}
+    t_roof = (c["indexer_flops"] / (fp8_peak * 1e12) + c["topk_bytes"] / (peaks["hbm_gbs"] * 1e9)
+              + c["attention_flops"] / (bf16_peak * 1e12))
+    roofline["step_frac"] = round(t_roof * 1e3 / step_ms, 4)
+    roofline["stages"] = {n: {"ms": round(float(stage_ms[i]), 4), "bound": per[n][0],
+                              "achieved": round(per[n][1], 2), "peak": per[n][2],
+                              "unit": per[n][3], "frac": round(per[n][1] / per[n][2], 4)}
+                          for i, n in enumerate(names)}
+
+    # ---- end to end through dsa_forward with host buffers
+    e2e = None
+    if not args.no_e2e and args.e2e_steps > 0:
+        e2e = run_e2e(dsa, wl, args, world, local, stream)
+
+    # ---- CPU baseline: the oracle, rank 0 at N=1 only
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        n_rows = max(8, min(64, 2 * oracle_threads()))
+        dt, desc = oracle_sample(wl, n_rows, seed=99)
+        cpu = {"value": round(n_rows / dt, 4), "unit": UNIT, "cores": oracle_threads(),
+               "kind": "oracle", "sample": desc, "seconds": round(dt, 2)}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8e4m3+bf16", "data": "synthetic",
+            "config": {"workload": f"{cfg.name} (one causal prefill per GPU)", "L": cfg.L,
+                       "H_I": H_I, "d_I": d_I, "H": H, "d_qk": 576, "d_v": 512, "k": wl.k,
+                       "global_batch_sequences": world, "parallelism": f"dp{world}",
+                       "l2": "flushed between steps (256 MiB write outside the timed events)"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": 3 * args.steps, "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(dsa, wl, args, world, local, stream):
+    names = ("q8", "q_scale", "w", "k8", "k_scale", "q", "kv", "cu_q", "cu_k")
+    host = {n: getattr(wl, n).cpu().pin_memory() for n in names}
+    dev = {n: torch.empty_like(getattr(wl, n)) for n in names}
+    H = wl.q.shape[1]
+    out_h = torch.empty((wl.T_q, H, 512), dtype=torch.bfloat16).pin_memory()
+    lse_h = torch.empty((wl.T_q, H), dtype=torch.float32).pin_memory()
+    out = torch.empty((wl.T_q, H, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((wl.T_q, H), dtype=torch.float32, device="cuda")
+    ws = torch.empty(dsa.dsa_forward_workspace_size(wl.T_q, wl.max_len_k, wl.k), dtype=torch.uint8,
+                     device="cuda")
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+
+    def one(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        for n in names:
+            dev[n].copy_(host[n], non_blocking=True)
+        dsa.dsa_forward(dev["q8"], dev["q_scale"], dev["w"], dev["k8"], dev["k_scale"], dev["q"],
+                        dev["kv"], dev["cu_q"], dev["cu_k"], wl.B, wl.max_len_q, wl.max_len_k,
+                        wl.k, wl.scale, out, lse, ws, stream=stream)
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+        if ev is not None:
+            ev[1].record(stream)
+
+    one()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.e2e_steps)]
+    for i in range(args.e2e_steps):
+        one(evs[i])
+    torch.cuda.synchronize()
+    ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": round(world * wl.T_q / (ms / 1e3), 1), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": round(ms, 3), "steps": args.e2e_steps, "api": "dsa_forward"}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    from sparse_attention_08_b200 import workloads as W
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    cfg = W.CONFIGS[args.config]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    wl = W.make_prefill(args.config, device=dev)
+    n_rows = max(4, oracle_threads())
+    for i in range(args.warmup):
+        oracle_sample(wl, max(1, n_rows // 4), seed=1000 + i)
+    secs = []
+    for i in range(args.steps):
+        dt, desc = oracle_sample(wl, n_rows, seed=i)
+        secs.append(dt)
+    step_s = float(np.mean(secs))
+    value = n_rows / step_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(step_s * 1e3, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{cfg.name} (one causal prefill)", "L": cfg.L, "k": cfg.k,
+                   "H": cfg.H, "H_I": cfg.H_I, "d_I": cfg.d_I,
+                   "step": f"{n_rows} sampled query rows per step"},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": oracle_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,183 @@
+/*
+ * dsa.h -- C ABI of libdsa.so, the B200 (sm_100a) hot path of DeepSeek Sparse
+ * Attention (DSA): lightning-indexer scores -> per-query top-k -> sparse
+ * attention in the MQA mode of MLA.
+ *
+ * The operation, as the pages state it:
+ *  - "DeepSeek V3.2 and the lightning indexer" (montana-research blog),
+ *    section "How the lightning indexer works": a few indexer heads score each
+ *    query against every earlier token as a weighted sum of ReLU'd dot
+ *    products, in FP8; each query keeps its 2,048 best entries; the main
+ *    attention runs over those only; DSA sits on the MQA mode of MLA, so one
+ *    latent serves all query heads and the selection is made per position.
+ *  - "DeepSeek-V3.2" (atlas.lewiswon.me), "Design overview": token-level
+ *    top-k with k = 2048, main attention cost O(L*k).
+ *  - "DeepSeek-V3.2 ... (introducing DSA)" (phantomic12 paper record): one
+ *    scalar indexer logit per (query, KV) pair; only the top-k are attended;
+ *    the indexer is a full-context pass, which is why it runs in FP8.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  Pointers marked (device) are CUDA device pointers owned by the caller; the
+ *  library allocates no device memory and keeps no pointer after returning.
+ *  All work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is
+ *  the legacy default stream) and nothing synchronises with the host, except
+ *  dsa_get_device_error().
+ *
+ *  Varlen batches: B sequences; cu_seqlens_q / cu_seqlens_k are (device)
+ *  int32 arrays of B+1 non-decreasing offsets.  Sequence b owns query rows
+ *  cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 and key rows cu_seqlens_k[b] ..
+ *  cu_seqlens_k[b+1]-1, with len_q <= len_k.  Its queries are the LAST len_q
+ *  positions of the sequence: local query i sits at absolute position
+ *  p = (len_k - len_q) + i and may use the sequence-local keys 0..p (causal,
+ *  self included).  Prefill: len_q = len_k.  Chunked prefill: len_q = chunk,
+ *  len_k = chunk end.  Decode: len_q = 1.
+ *  max_len_q / max_len_k bound the per-sequence lengths; total_q / total_k
+ *  are cu_seqlens_q[B] / cu_seqlens_k[B] (the caller knows them; the host
+ *  code never reads device memory).
+ *
+ *  Layouts are row-major and contiguous unless a leading dimension is given.
+ *  Every pointer must be 16-byte aligned (DSA_ERR_ALIGNMENT otherwise).
+ *
+ *  Errors: each call validates its arguments before launching anything and
+ *  returns a status; CUDA launch errors map to DSA_ERR_CUDA.  Kernels bound
+ *  every wait; a wait that runs out sets a device error word and the kernel
+ *  returns early.  dsa_get_device_error() reads and clears that word.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1, /* a size, count or pointer is out of range / NULL */
+  DSA_ERR_UNSUPPORTED = 2, /* valid but outside the shapes this build supports */
+  DSA_ERR_ALIGNMENT = 3,   /* a pointer or stride breaks the 16-byte rule */
+  DSA_ERR_WORKSPACE = 4,   /* workspace NULL or smaller than required */
+  DSA_ERR_CUDA = 5,        /* a CUDA runtime / driver call failed */
+  DSA_ERR_TIMEOUT = 6,     /* a kernel gave up on a bounded wait */
+  DSA_ERR_BOUNDS = 7       /* a kernel found an index outside its tensor */
+} dsa_status_t;
+
+/*
+ * Lightning-indexer scores (blog, "How the lightning indexer works"):
+ *
+ *   logits[q_row, s] = k_scale[k_row] *
+ *                      sum_j (w[q_row,j] * q_scale[q_row,j]) * ReLU(q8[q_row,j,:] . k8[k_row,:])
+ *
+ * for every causal pair (s <= p), where q_row is the global query row, s the
+ * sequence-local key position and k_row = cu_seqlens_k[b] + s.  This equals
+ * sum_j w * ReLU(qhat . khat) on the dequantised vectors qhat = q8 * q_scale,
+ * khat = k8 * k_scale whenever the scales are positive.
+ *
+ *  q_fp8    (device) e4m3 bytes [total_q, H_I, d_I]
+ *  q_scale  (device) f32 [total_q, H_I]   (> 0; a per-token scale is replicated)
+ *  w        (device) f32 [total_q, H_I]   indexer head weights (any sign)
+ *  k_fp8    (device) e4m3 bytes [total_k, d_I]  (one head, shared by all H_I)
+ *  k_scale  (device) f32 [total_k]        (> 0)
+ *  logits   (device) f32, row q_row at logits + q_row * ld_logits, column s;
+ *           ld_logits >= max_len_k and a multiple of 4.  Only entries with
+ *           s <= p are written; the rest are left untouched.
+ *  Supported: d_I in {64, 128}; H_I in {4, 8, 16, 32, 64, 128}.
+ *  Arithmetic: FP8 products accumulated by the tensor core, fp32 epilogue.
+ */
+DSA_API dsa_status_t dsa_indexer_logits(const void* q_fp8, const float* q_scale, const float* w,
+                                const void* k_fp8, const float* k_scale,
+                                const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
+                                int max_len_q, int max_len_k, int64_t total_q, int64_t total_k,
+                                int H_I, int d_I, float* logits, int64_t ld_logits, void* stream);
+
+/*
+ * Per-query top-k (blog, "How the lightning indexer works"; atlas,
+ * "Design overview": token-level selection of the k best entries per query).
+ *
+ * For each query row, reads logits[q_row, 0..p] and writes to idx_out[q_row,
+ * 0..k) the sequence-local positions of the min(k, p+1) largest scores in
+ * ascending position order, padded with -1.  Ties go to the lower position;
+ * -0.0 and +0.0 are equal.  NaN scores are not supported.
+ *
+ *  logits   (device) f32, layout as produced by dsa_indexer_logits
+ *  idx_out  (device) int32 [total_q, k]
+ *  val_out  (device, nullable) f32 [total_q, k]: the selected scores (NaN in
+ *           padding slots)
+ *  Supported: 1 <= k <= 4096, max_len_k <= 2^24.
+ */
+DSA_API dsa_status_t dsa_topk(const float* logits, int64_t ld_logits, const int32_t* cu_seqlens_q,
+                      const int32_t* cu_seqlens_k, int B, int max_len_q, int max_len_k,
+                      int64_t total_q, int k, int32_t* idx_out, float* val_out, void* stream);
+
+/*
+ * Sparse attention in the MQA mode of MLA (blog, "How the lightning indexer
+ * works": each selected latent is shared by all query heads; atlas,
+ * "Inference efficiency": attention touches only the selected latents).
+ *
+ *   out[q_row, h, :] = sum_{s in S} softmax_s(sm_scale * q[q_row,h,:] . kv[k_row(s),:])
+ *                                  * kv[k_row(s), 0:d_v]
+ *   lse[q_row, h]    = log sum_{s in S} exp(sm_scale * q[q_row,h,:] . kv[k_row(s),:])
+ *
+ * S is the set of entries among the FIRST min(k, p+1) of idx[q_row, :] that
+ * satisfy 0 <= s <= p; other entries are skipped (dsa_topk fills exactly that
+ * prefix).  A row with an empty S gets out = 0 and lse = -inf.
+ *
+ *  q        (device) bf16 [total_q, H, d_qk]
+ *  kv       (device) bf16 [total_k, d_qk]; the first d_v dims are the value
+ *  idx      (device) int32 [total_q, k]
+ *  out      (device) bf16 [total_q, H, d_v]
+ *  lse      (device, nullable) f32 [total_q, H] (natural log)
+ *  Supported: d_qk = 576, d_v = 512, H in {16, 32} or a multiple of 64 up to
+ *  256, 1 <= k <= 4096.
+ *  Arithmetic: bf16 tensor-core products, fp32 accumulation and softmax.
+ */
+DSA_API dsa_status_t dsa_sparse_mla_fwd(const void* q, const void* kv, const int32_t* idx,
+                                const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
+                                int max_len_q, int max_len_k, int64_t total_q, int64_t total_k,
+                                int H, int d_qk, int d_v, int k, float sm_scale, void* out,
+                                float* lse, void* stream);
+
+/*
+ * The whole path on one stream: dsa_indexer_logits -> dsa_topk ->
+ * dsa_sparse_mla_fwd, with the scores and indices kept in the caller's
+ * workspace (size from dsa_forward_workspace_size).  idx_out (nullable)
+ * receives a copy of the selected indices [total_q, k].
+ */
+DSA_API dsa_status_t dsa_forward(const void* q_fp8, const float* q_scale, const float* w,
+                         const void* k_fp8, const float* k_scale, const void* q, const void* kv,
+                         const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
+                         int max_len_q, int max_len_k, int64_t total_q, int64_t total_k, int H_I,
+                         int d_I, int H, int d_qk, int d_v, int k, float sm_scale, void* out,
+                         float* lse, int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/* Bytes of workspace dsa_forward needs: an f32 score matrix [total_q,
+ * round_up(max_len_k, 4)] plus an int32 index matrix [total_q, k], each
+ * 256-byte aligned.  Returns 0 for invalid sizes. */
+DSA_API size_t dsa_forward_workspace_size(int64_t total_q, int max_len_k, int k);
+
+/* Static text for a status code (never NULL). */
+DSA_API const char* dsa_status_string(dsa_status_t status);
+
+/* Synchronises `stream`, then reads and clears the device error word that
+ * the kernels set on a timed-out wait (DSA_ERR_TIMEOUT) or a bounds failure
+ * (DSA_ERR_BOUNDS).  Returns DSA_OK if it was clear. */
+DSA_API dsa_status_t dsa_get_device_error(void* stream);
+
+/* Library version, "major.minor.patch". */
+DSA_API const char* dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

@@ -61,6 +61,14 @@ def _load():
         lib.oracle_forward.restype = i32
         lib.oracle_forward.argtypes = [P, P, P, P, P, P, P, i64, i64, i32, i32, i32, i32, i32, i32,
                                        ctypes.c_double, P, i64, P, P, P]
+        lib.oracle_forward_at.restype = i32
+        lib.oracle_forward_at.argtypes = [P, P, P, P, P, P, P, P, i64, i64, i32, i32, i32, i32, i32,
+                                          i32, ctypes.c_double, P, P, P]
+        lib.oracle_indexer_at.restype = i32
+        lib.oracle_indexer_at.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, P, i64]
+        lib.oracle_sparse_mla_at.restype = i32
+        lib.oracle_sparse_mla_at.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, i32,
+                                             ctypes.c_double, P, P]
         lib.oracle_num_threads.restype = i32
         lib.oracle_num_threads.argtypes = []
         _lib = lib
@@ -176,3 +184,64 @@ def forward(q8, q_scale, w, k8, k_scale, q_bits, kv_bits, k, scale, d_v=512, row
     if rc != 0:
         raise ValueError("oracle_forward: bad arguments")
     return idx, out, lse
+
+
+def forward_at(q8, q_scale, w, k8, k_scale, q_bits, kv_bits, pos, k, scale, d_v=512):
+    """The whole path for query rows given with their positions: row r of the
+    query-side arrays sits at position pos[r] of the sequence whose keys are
+    k8 / k_scale / kv_bits.  Returns (idx [R, k], out [R, H, d_v], lse [R, H])."""
+    q8 = _c(q8, np.uint8)
+    k8 = _c(k8, np.uint8)
+    q_bits = _c(q_bits, np.uint16)
+    kv_bits = _c(kv_bits, np.uint16)
+    pos = _c(pos, np.int64)
+    R, H_I, d_I = q8.shape
+    n_k = k8.shape[0]
+    _, H, d_qk = q_bits.shape
+    idx = np.empty((R, k), dtype=np.int32)
+    out = np.empty((R, H, d_v), dtype=np.float64)
+    lse = np.empty((R, H), dtype=np.float64)
+    rc = _load().oracle_forward_at(_ptr(q8), _ptr(_c(q_scale, np.float32)), _ptr(_c(w, np.float32)),
+                                   _ptr(k8), _ptr(_c(k_scale, np.float32)), _ptr(q_bits),
+                                   _ptr(kv_bits), _ptr(pos), R, n_k, H_I, d_I, H, d_qk, d_v, k,
+                                   float(scale), _ptr(idx), _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_forward_at: bad arguments")
+    return idx, out, lse
+
+
+def indexer_at(q8, q_scale, w, k8, k_scale, pos):
+    """Indexer scores of query rows at explicit positions: row r of q8 /
+    q_scale / w sits at position pos[r].  Returns float64 [R, n_k], NaN where
+    s > pos[r]."""
+    q8 = _c(q8, np.uint8)
+    k8 = _c(k8, np.uint8)
+    pos = _c(pos, np.int64)
+    R, H_I, d_I = q8.shape
+    n_k = k8.shape[0]
+    out = np.full((R, n_k), np.nan, dtype=np.float64)
+    rc = _load().oracle_indexer_at(_ptr(q8), _ptr(_c(q_scale, np.float32)), _ptr(_c(w, np.float32)),
+                                   _ptr(k8), _ptr(_c(k_scale, np.float32)), _ptr(pos), R, n_k, H_I,
+                                   d_I, _ptr(out), n_k)
+    if rc != 0:
+        raise ValueError("oracle_indexer_at: bad arguments")
+    return out
+
+
+def sparse_mla_at(q_bits, kv_bits, idx, pos, scale, d_v=512):
+    """Sparse attention of query rows at explicit positions pos[r] (idx row r
+    is row r's selection).  Returns (out [R, H, d_v], lse [R, H])."""
+    q_bits = _c(q_bits, np.uint16)
+    kv_bits = _c(kv_bits, np.uint16)
+    idx = _c(idx, np.int32)
+    pos = _c(pos, np.int64)
+    R, H, d_qk = q_bits.shape
+    n_k = kv_bits.shape[0]
+    k = idx.shape[1]
+    out = np.empty((R, H, d_v), dtype=np.float64)
+    lse = np.empty((R, H), dtype=np.float64)
+    rc = _load().oracle_sparse_mla_at(_ptr(q_bits), _ptr(kv_bits), _ptr(idx), _ptr(pos), R, n_k, H,
+                                      d_qk, d_v, k, float(scale), _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_sparse_mla_at: bad arguments")
+    return out, lse

@@ -310,6 +310,98 @@ int oracle_forward(const uint8_t* q8, const float* q_scale, const float* w, cons
   return bad ? -1 : 0;
 }
 
+/* The whole path for query rows given with their positions: row r of the
+ * query-side arrays (q8, q_scale, w, q) sits at position pos[r] < n_k of a
+ * sequence whose keys are k8 / k_scale / kv.  Same arithmetic as
+ * oracle_forward; used to evaluate sampled rows of a long sequence without
+ * materialising the other query rows. */
+int oracle_forward_at(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8,
+                      const float* k_scale, const uint16_t* q, const uint16_t* kv,
+                      const int64_t* pos, int64_t n_rows, int64_t n_k, int H_I, int d_I, int H,
+                      int d_qk, int d_v, int k, double scale, int32_t* idx_out, double* out,
+                      double* lse) {
+  if (k <= 0 || d_v > d_qk || H <= 0 || H_I <= 0 || d_I <= 0 || !pos) return -1;
+  int bad = 0;
+#pragma omp parallel
+  {
+    double* scores = (double*)malloc(sizeof(double) * (size_t)(n_k > 0 ? n_k : 1));
+    scored_t* scratch = (scored_t*)malloc(sizeof(scored_t) * (size_t)(n_k > 0 ? n_k : 1));
+    int32_t* idx = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+    int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+    double* x = (double*)malloc(sizeof(double) * (size_t)k);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; ++r) {
+      int64_t p = pos[r];
+      if (p < 0 || p >= n_k || !scores || !scratch || !idx || !sel || !x) {
+        bad = 1;
+        continue;
+      }
+      for (int64_t s = 0; s <= p; ++s)
+        scores[s] = indexer_score(q8, q_scale, w, k8, k_scale, r, s, H_I, d_I);
+      topk_row(scores, p + 1, k, scratch, idx);
+      if (idx_out) memcpy(idx_out + r * (int64_t)k, idx, sizeof(int32_t) * (size_t)k);
+      int64_t n_sel = valid_entries(idx, k, p, sel);
+      attend_row(q, kv, sel, n_sel, r, H, d_qk, d_v, scale, out + r * (int64_t)H * d_v,
+                 lse + r * (int64_t)H, x);
+    }
+    free(scores);
+    free(scratch);
+    free(idx);
+    free(sel);
+    free(x);
+  }
+  return bad ? -1 : 0;
+}
+
+/* Indexer scores of query rows given with their positions: row r of q8 /
+ * q_scale / w sits at position pos[r] < n_k; out[r * ld_out + s] = I[r, s]
+ * for s <= pos[r]. */
+int oracle_indexer_at(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8,
+                      const float* k_scale, const int64_t* pos, int64_t n_rows, int64_t n_k,
+                      int H_I, int d_I, double* out, int64_t ld_out) {
+  if (H_I <= 0 || d_I <= 0 || ld_out < n_k || !pos) return -1;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    int64_t p = pos[r];
+    if (p < 0 || p >= n_k) {
+      bad = 1;
+      continue;
+    }
+    for (int64_t s = 0; s <= p; ++s)
+      out[r * ld_out + s] = indexer_score(q8, q_scale, w, k8, k_scale, r, s, H_I, d_I);
+  }
+  return bad ? -1 : 0;
+}
+
+/* Sparse attention of query rows given with their positions (row r of q at
+ * position pos[r]; idx row r is its selection). */
+int oracle_sparse_mla_at(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
+                         const int64_t* pos, int64_t n_rows, int64_t n_k, int H, int d_qk,
+                         int d_v, int k, double scale, double* out, double* lse) {
+  if (k <= 0 || d_v > d_qk || H <= 0 || !pos) return -1;
+  int bad = 0;
+#pragma omp parallel
+  {
+    int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+    double* x = (double*)malloc(sizeof(double) * (size_t)k);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; ++r) {
+      int64_t p = pos[r];
+      if (p < 0 || p >= n_k || !sel || !x) {
+        bad = 1;
+        continue;
+      }
+      int64_t n_sel = valid_entries(idx + r * (int64_t)k, k, p, sel);
+      attend_row(q, kv, sel, n_sel, r, H, d_qk, d_v, scale, out + r * (int64_t)H * d_v,
+                 lse + r * (int64_t)H, x);
+    }
+    free(sel);
+    free(x);
+  }
+  return bad ? -1 : 0;
+}
+
 /* Threads OpenMP will use (reported beside the CPU baseline). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

@@ -1,0 +1,205 @@
+"""B200-native DeepSeek Sparse Attention (DSA) hot path.
+
+The compute lives in ``libdsa.so`` (CUDA for sm_100a, C ABI in
+``include/dsa.h``); this module only marshals torch tensors into that ABI.
+Every function has the name of its C entry point and takes device tensors
+plus the stream it should run on (default: torch's current stream).  There is
+no CPU path: if the library is missing, importing the binding fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "DSAError", "lib_path", "load", "dsa_version", "dsa_status_string",
+    "dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward",
+    "dsa_forward_workspace_size", "dsa_get_device_error", "EXPORTED",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libdsa.so")
+_lib = None
+
+# Every symbol include/dsa.h declares.
+EXPORTED = (
+    "dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward",
+    "dsa_forward_workspace_size", "dsa_status_string", "dsa_get_device_error", "dsa_version",
+)
+
+STATUS = {
+    0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "DSA_ERR_ALIGNMENT",
+    4: "DSA_ERR_WORKSPACE", 5: "DSA_ERR_CUDA", 6: "DSA_ERR_TIMEOUT", 7: "DSA_ERR_BOUNDS",
+}
+
+
+class DSAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {STATUS.get(self.status, self.status)} "
+                         f"({dsa_status_string(self.status)})")
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Loads libdsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                          "`python -m sparse_attention_08_b200._build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I, I64, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+    lib.dsa_indexer_logits.argtypes = [P, P, P, P, P, P, P, I, I, I, I64, I64, I, I, P, I64, P]
+    lib.dsa_topk.argtypes = [P, I64, P, P, I, I, I, I64, I, P, P, P]
+    lib.dsa_sparse_mla_fwd.argtypes = [P, P, P, P, P, I, I, I, I64, I64, I, I, I, I, F, P, P, P]
+    lib.dsa_forward.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I64, I64, I, I, I, I, I, I, F,
+                                P, P, P, P, ctypes.c_size_t, P]
+    for name in ("dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward"):
+        getattr(lib, name).restype = I
+    lib.dsa_forward_workspace_size.argtypes = [I64, I, I]
+    lib.dsa_forward_workspace_size.restype = ctypes.c_size_t
+    lib.dsa_status_string.argtypes = [I]
+    lib.dsa_status_string.restype = ctypes.c_char_p
+    lib.dsa_get_device_error.argtypes = [P]
+    lib.dsa_get_device_error.restype = I
+    lib.dsa_version.argtypes = []
+    lib.dsa_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def dsa_version() -> str:
+    return load().dsa_version().decode()
+
+
+def dsa_status_string(status: int) -> str:
+    return load().dsa_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise DSAError(rc, where)
+
+
+def _need(t, dtype, name, ndim=None):
+    import torch
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims")
+    del torch
+
+
+def dsa_indexer_logits(q_fp8, q_scale, w, k_fp8, k_scale, cu_seqlens_q, cu_seqlens_k, B,
+                       max_len_q, max_len_k, logits, ld_logits=None, stream=None):
+    """Indexer scores into logits (f32, row stride ld_logits).  q_fp8 / k_fp8
+    are uint8 (or float8_e4m3fn) tensors [T_q, H_I, d_I] / [T_k, d_I]."""
+    import torch
+    q8 = q_fp8.view(torch.uint8) if q_fp8.dtype == torch.float8_e4m3fn else q_fp8
+    k8 = k_fp8.view(torch.uint8) if k_fp8.dtype == torch.float8_e4m3fn else k_fp8
+    _need(q8, torch.uint8, "q_fp8", 3)
+    _need(k8, torch.uint8, "k_fp8", 2)
+    _need(q_scale, torch.float32, "q_scale")
+    _need(w, torch.float32, "w")
+    _need(k_scale, torch.float32, "k_scale")
+    _need(cu_seqlens_q, torch.int32, "cu_seqlens_q")
+    _need(cu_seqlens_k, torch.int32, "cu_seqlens_k")
+    if ld_logits is None:
+        ld_logits = logits.stride(0)
+    T_q, H_I, d_I = q8.shape
+    rc = load().dsa_indexer_logits(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale),
+                                   _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(B), int(max_len_q),
+                                   int(max_len_k), int(T_q), int(k8.shape[0]), int(H_I), int(d_I),
+                                   _ptr(logits), int(ld_logits), _stream(stream))
+    _check(rc, "dsa_indexer_logits")
+
+
+def dsa_topk(logits, cu_seqlens_q, cu_seqlens_k, B, max_len_q, max_len_k, k, idx_out,
+             val_out=None, ld_logits=None, total_q=None, stream=None):
+    import torch
+    _need(idx_out, torch.int32, "idx_out", 2)
+    _need(val_out, torch.float32, "val_out", 2)
+    if logits.dtype != torch.float32 or not logits.is_cuda:
+        raise ValueError("logits must be a CUDA float32 tensor")
+    if ld_logits is None:
+        ld_logits = logits.stride(0)
+    if total_q is None:
+        total_q = idx_out.shape[0]
+    rc = load().dsa_topk(_ptr(logits), int(ld_logits), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+                         int(B), int(max_len_q), int(max_len_k), int(total_q), int(k),
+                         _ptr(idx_out), _ptr(val_out), _stream(stream))
+    _check(rc, "dsa_topk")
+
+
+def dsa_sparse_mla_fwd(q, kv, idx, cu_seqlens_q, cu_seqlens_k, B, max_len_q, max_len_k,
+                       sm_scale, out, lse=None, stream=None):
+    import torch
+    _need(q, torch.bfloat16, "q", 3)
+    _need(kv, torch.bfloat16, "kv", 2)
+    _need(idx, torch.int32, "idx", 2)
+    _need(out, torch.bfloat16, "out", 3)
+    _need(lse, torch.float32, "lse", 2)
+    T_q, H, d_qk = q.shape
+    rc = load().dsa_sparse_mla_fwd(_ptr(q), _ptr(kv), _ptr(idx), _ptr(cu_seqlens_q),
+                                   _ptr(cu_seqlens_k), int(B), int(max_len_q), int(max_len_k),
+                                   int(T_q), int(kv.shape[0]), int(H), int(d_qk),
+                                   int(out.shape[2]), int(idx.shape[1]), float(sm_scale),
+                                   _ptr(out), _ptr(lse), _stream(stream))
+    _check(rc, "dsa_sparse_mla_fwd")
+
+
+def dsa_forward_workspace_size(total_q, max_len_k, k) -> int:
+    return int(load().dsa_forward_workspace_size(int(total_q), int(max_len_k), int(k)))
+
+
+def dsa_forward(q_fp8, q_scale, w, k_fp8, k_scale, q, kv, cu_seqlens_q, cu_seqlens_k, B,
+                max_len_q, max_len_k, k, sm_scale, out, lse, workspace, idx_out=None,
+                stream=None):
+    import torch
+    q8 = q_fp8.view(torch.uint8) if q_fp8.dtype == torch.float8_e4m3fn else q_fp8
+    k8 = k_fp8.view(torch.uint8) if k_fp8.dtype == torch.float8_e4m3fn else k_fp8
+    _need(q8, torch.uint8, "q_fp8", 3)
+    _need(k8, torch.uint8, "k_fp8", 2)
+    _need(q, torch.bfloat16, "q", 3)
+    _need(kv, torch.bfloat16, "kv", 2)
+    _need(out, torch.bfloat16, "out", 3)
+    _need(lse, torch.float32, "lse", 2)
+    _need(idx_out, torch.int32, "idx_out", 2)
+    T_q, H_I, d_I = q8.shape
+    _, H, d_qk = q.shape
+    rc = load().dsa_forward(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale), _ptr(q),
+                            _ptr(kv), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(B),
+                            int(max_len_q), int(max_len_k), int(T_q), int(k8.shape[0]), int(H_I),
+                            int(d_I), int(H), int(d_qk), int(out.shape[2]), int(k),
+                            float(sm_scale), _ptr(out), _ptr(lse), _ptr(idx_out),
+                            _ptr(workspace), int(workspace.numel() * workspace.element_size()),
+                            _stream(stream))
+    _check(rc, "dsa_forward")
+
+
+def dsa_get_device_error(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device error
+    status: 0 = DSA_OK, 6 = DSA_ERR_TIMEOUT, 7 = DSA_ERR_BOUNDS."""
+    return int(load().dsa_get_device_error(_stream(stream)))

@@ -1,0 +1,302 @@
+// api.cu -- the C ABI of libdsa.so (declared in include/dsa.h): argument
+// validation, TMA tensor-map encoding, the device error word, and the
+// sequencing of the three stages on the caller's stream.
+//
+// The library allocates no device memory: the error word below is a static
+// __device__ variable of the module, and every buffer comes from the caller.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "dsa.h"
+#include "internal.h"
+
+namespace {
+
+__device__ unsigned g_dsa_err[2];  // [0] sticky error bits, [1] newest failed launch generation
+
+std::atomic<unsigned> g_generation{1};
+
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+  unsigned* err = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+dsa_status_t device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dsa_err) != cudaSuccess) return DSA_ERR_CUDA;
+    d.err = static_cast<unsigned*>(p);
+    d.ready = true;
+  }
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return DSA_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  *out = &d;
+  return DSA_OK;
+}
+
+dsa::DevErr next_err(const DeviceInfo* d) {
+  dsa::DevErr e;
+  e.word = d->err;
+  e.gen = g_generation.fetch_add(1);
+  return e;
+}
+
+// Row-major 2D tensor [rows, cols] of `elem` bytes per element, box of
+// box_rows x box_cols elements.
+dsa_status_t encode_2d(CUtensorMap* m, CUtensorMapDataType dtype, const void* base, uint64_t rows,
+                       uint64_t cols, uint64_t elem, uint32_t box_rows, uint32_t box_cols,
+                       CUtensorMapSwizzle swz) {
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * elem};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+dsa_status_t check_varlen(const int32_t* cu_q, const int32_t* cu_k, int B, int max_len_q,
+                          int max_len_k, int64_t total_q, int64_t total_k) {
+  if (!cu_q || !cu_k || B < 0 || max_len_q < 0 || max_len_k < 0 || total_q < 0 || total_k < 0)
+    return DSA_ERR_INVALID_ARG;
+  if (max_len_q > max_len_k) return DSA_ERR_INVALID_ARG;
+  if (total_q > (int64_t)B * max_len_q || total_k > (int64_t)B * max_len_k)
+    return DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
+dsa_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+
+bool indexer_shape_ok(int H_I, int d_I) {
+  const bool h = H_I == 4 || H_I == 8 || H_I == 16 || H_I == 32 || H_I == 64 || H_I == 128;
+  return h && (d_I == 64 || d_I == 128);
+}
+
+bool mla_heads_ok(int H) { return H == 16 || H == 32 || (H % 64 == 0 && H >= 64 && H <= 256); }
+
+}  // namespace
+
+extern "C" {
+
+const char* dsa_version(void) { return "0.1.0"; }
+
+const char* dsa_status_string(dsa_status_t s) {
+  switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case DSA_ERR_ALIGNMENT: return "pointer or stride not 16-byte aligned";
+    case DSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_TIMEOUT: return "device wait timed out";
+    case DSA_ERR_BOUNDS: return "device bounds check failed";
+  }
+  return "unknown status";
+}
+
+dsa_status_t dsa_indexer_logits(const void* q_fp8, const float* q_scale, const float* w,
+                                const void* k_fp8, const float* k_scale,
+                                const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
+                                int max_len_q, int max_len_k, int64_t total_q, int64_t total_k,
+                                int H_I, int d_I, float* logits, int64_t ld_logits, void* stream) {
+  dsa_status_t st = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_len_q, max_len_k, total_q,
+                                 total_k);
+  if (st != DSA_OK) return st;
+  if (!q_fp8 || !q_scale || !w || !k_fp8 || !k_scale || !logits) return DSA_ERR_INVALID_ARG;
+  if (!indexer_shape_ok(H_I, d_I)) return DSA_ERR_UNSUPPORTED;
+  if (ld_logits < max_len_k || ld_logits < 1) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_fp8) || !aligned16(k_fp8) || !aligned16(logits) || (ld_logits % 4) != 0)
+    return DSA_ERR_ALIGNMENT;
+  if (total_q * H_I >= (int64_t(1) << 31) || total_k >= (int64_t(1) << 31))
+    return DSA_ERR_UNSUPPORTED;
+  if (total_q == 0 || total_k == 0 || B == 0) return DSA_OK;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != DSA_OK) return st;
+  const CUtensorMapSwizzle swz =
+      d_I == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUtensorMap tq, tk;
+  if ((st = encode_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_fp8, total_q * H_I, d_I, 1, 256, d_I,
+                      swz)) != DSA_OK)
+    return st;
+  if ((st = encode_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, k_fp8, total_k, d_I, 1, 128, d_I,
+                      swz)) != DSA_OK)
+    return st;
+  dsa::IndexerArgs a;
+  a.q_scale = q_scale;
+  a.w = w;
+  a.k_scale = k_scale;
+  a.cu_q = cu_seqlens_q;
+  a.cu_k = cu_seqlens_k;
+  a.B = B;
+  a.max_len_q = max_len_q;
+  a.max_len_k = max_len_k;
+  a.H_I = H_I;
+  a.d_I = d_I;
+  a.logits = logits;
+  a.ld = ld_logits;
+  return from_cuda(dsa::launch_indexer(tq, tk, a, dev->num_sms, next_err(dev),
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+dsa_status_t dsa_topk(const float* logits, int64_t ld_logits, const int32_t* cu_seqlens_q,
+                      const int32_t* cu_seqlens_k, int B, int max_len_q, int max_len_k,
+                      int64_t total_q, int k, int32_t* idx_out, float* val_out, void* stream) {
+  dsa_status_t st =
+      check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_len_q, max_len_k, total_q, 0);
+  if (st != DSA_OK) return st;
+  if (!logits || !idx_out) return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > 4096) return DSA_ERR_UNSUPPORTED;
+  if (max_len_k > (1 << 24)) return DSA_ERR_UNSUPPORTED;
+  if (ld_logits < max_len_k || ld_logits < 1) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(logits) || !aligned16(idx_out) || (val_out && !aligned16(val_out)))
+    return DSA_ERR_ALIGNMENT;
+  if (total_q >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
+  if (total_q == 0 || B == 0) return DSA_OK;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != DSA_OK) return st;
+  dsa::TopkArgs a;
+  a.logits = logits;
+  a.ld = ld_logits;
+  a.cu_q = cu_seqlens_q;
+  a.cu_k = cu_seqlens_k;
+  a.B = B;
+  a.max_len_q = max_len_q;
+  a.max_len_k = max_len_k;
+  a.total_q = total_q;
+  a.k = k;
+  a.idx = idx_out;
+  a.val = val_out;
+  return from_cuda(dsa::launch_topk(a, next_err(dev), static_cast<cudaStream_t>(stream)));
+}
+
+dsa_status_t dsa_sparse_mla_fwd(const void* q, const void* kv, const int32_t* idx,
+                                const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
+                                int max_len_q, int max_len_k, int64_t total_q, int64_t total_k,
+                                int H, int d_qk, int d_v, int k, float sm_scale, void* out,
+                                float* lse, void* stream) {
+  dsa_status_t st = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_len_q, max_len_k, total_q,
+                                 total_k);
+  if (st != DSA_OK) return st;
+  if (!q || !kv || !idx || !out) return DSA_ERR_INVALID_ARG;
+  if (d_qk != 576 || d_v != 512 || !mla_heads_ok(H) || k < 1 || k > 4096)
+    return DSA_ERR_UNSUPPORTED;
+  if (!(sm_scale > 0.f) || sm_scale != sm_scale) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(idx) || !aligned16(out) ||
+      (lse && !aligned16(lse)))
+    return DSA_ERR_ALIGNMENT;
+  const int64_t groups = (H + 63) / 64;
+  if (total_q * H >= (int64_t(1) << 31) || total_q * groups >= (int64_t(1) << 31) ||
+      total_k >= (int64_t(1) << 31))
+    return DSA_ERR_UNSUPPORTED;
+  if (total_q == 0 || B == 0) return DSA_OK;
+  if (total_k == 0) return DSA_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != DSA_OK) return st;
+  CUtensorMap tq, tkv;
+  if ((st = encode_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, total_q * H, 576, 2, 64, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != DSA_OK)
+    return st;
+  if ((st = encode_2d(&tkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kv, total_k, 576, 2, 1, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != DSA_OK)
+    return st;
+  dsa::MlaArgs a;
+  a.idx = idx;
+  a.cu_q = cu_seqlens_q;
+  a.cu_k = cu_seqlens_k;
+  a.B = B;
+  a.max_len_q = max_len_q;
+  a.max_len_k = max_len_k;
+  a.total_q = total_q;
+  a.total_k = total_k;
+  a.H = H;
+  a.k = k;
+  a.sm_scale = sm_scale;
+  a.out = out;
+  a.lse = lse;
+  return from_cuda(
+      dsa::launch_sparse_mla(tq, tkv, a, next_err(dev), static_cast<cudaStream_t>(stream)));
+}
+
+size_t dsa_forward_workspace_size(int64_t total_q, int max_len_k, int k) {
+  if (total_q < 0 || max_len_k < 0 || k < 1) return 0;
+  const int64_t ld = (static_cast<int64_t>(max_len_k) + 3) / 4 * 4;
+  const int64_t logits = (total_q * ld * 4 + 255) / 256 * 256;
+  const int64_t idx = (total_q * static_cast<int64_t>(k) * 4 + 255) / 256 * 256;
+  return static_cast<size_t>(logits + idx);
+}
+
+dsa_status_t dsa_forward(const void* q_fp8, const float* q_scale, const float* w,
+                         const void* k_fp8, const float* k_scale, const void* q, const void* kv,
+                         const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
+                         int max_len_q, int max_len_k, int64_t total_q, int64_t total_k, int H_I,
+                         int d_I, int H, int d_qk, int d_v, int k, float sm_scale, void* out,
+                         float* lse, int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  dsa_status_t st = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_len_q, max_len_k, total_q,
+                                 total_k);
+  if (st != DSA_OK) return st;
+  if (!indexer_shape_ok(H_I, d_I)) return DSA_ERR_UNSUPPORTED;
+  if (d_qk != 576 || d_v != 512 || !mla_heads_ok(H) || k < 1 || k > 4096)
+    return DSA_ERR_UNSUPPORTED;
+  const size_t need = dsa_forward_workspace_size(total_q, max_len_k, k);
+  if (!workspace || workspace_bytes < need) return DSA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return DSA_ERR_ALIGNMENT;
+  if (total_q == 0 || B == 0) return DSA_OK;
+  const int64_t ld = (static_cast<int64_t>(max_len_k) + 3) / 4 * 4;
+  float* logits = static_cast<float*>(workspace);
+  int32_t* idx = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) +
+                                            (total_q * ld * 4 + 255) / 256 * 256);
+  if (idx_out) idx = idx_out;
+  st = dsa_indexer_logits(q_fp8, q_scale, w, k_fp8, k_scale, cu_seqlens_q, cu_seqlens_k, B,
+                          max_len_q, max_len_k, total_q, total_k, H_I, d_I, logits, ld, stream);
+  if (st != DSA_OK) return st;
+  st = dsa_topk(logits, ld, cu_seqlens_q, cu_seqlens_k, B, max_len_q, max_len_k, total_q, k, idx,
+                nullptr, stream);
+  if (st != DSA_OK) return st;
+  return dsa_sparse_mla_fwd(q, kv, idx, cu_seqlens_q, cu_seqlens_k, B, max_len_q, max_len_k,
+                            total_q, total_k, H, d_qk, d_v, k, sm_scale, out, lse, stream);
+}
+
+dsa_status_t dsa_get_device_error(void* stream) {
+  DeviceInfo* dev = nullptr;
+  dsa_status_t st = device_info(&dev);
+  if (st != DSA_OK) return st;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSA_ERR_CUDA;
+  unsigned bits = 0;
+  if (cudaMemcpyFromSymbol(&bits, g_dsa_err, sizeof(unsigned)) != cudaSuccess) return DSA_ERR_CUDA;
+  if (bits == 0) return DSA_OK;
+  const unsigned zero = 0;
+  if (cudaMemcpyToSymbol(g_dsa_err, &zero, sizeof(unsigned)) != cudaSuccess) return DSA_ERR_CUDA;
+  if (bits & dsa::kErrTimeout) return DSA_ERR_TIMEOUT;
+  return DSA_ERR_BOUNDS;
+}
+
+}  // extern "C"

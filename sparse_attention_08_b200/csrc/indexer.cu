@@ -1,0 +1,361 @@
+// indexer.cu -- lightning-indexer scores on sm_100a.
+//
+// What it computes ("DeepSeek V3.2 and the lightning indexer", section "How
+// the lightning indexer works": a few indexer heads score every query against
+// each earlier token as a weighted sum of ReLU'd dot products, in FP8):
+//
+//   logits[t, s] = k_scale[s] * sum_j (w[t,j] * q_scale[t,j]) * ReLU(q8[t,j,:] . k8[s,:])
+//
+// for all causal pairs s <= p(t).
+//
+// How: the dot products form one dense FP8 contraction per tile,
+//   D[s, (t,j)] = sum_d k8[s,d] * q8[t,j,d],     M = 128 keys, N = 256 = QPT*H_I,
+// issued as tcgen05.mma kind::f8f6f4 (e4m3 x e4m3 -> f32) from TMA-fed,
+// 128/64-byte-swizzled shared-memory tiles into a double-buffered TMEM
+// accumulator.  Four epilogue warps own one key (TMEM lane) each and fold
+// ReLU, the (w * q_scale) head weights, the k_scale multiply and the causal
+// mask into the read-out, so no per-head score ever leaves the SM.
+//
+// Work items: (sequence, group of QPT queries, chunk of KB_PER_ITEM key
+// blocks) on a persistent grid of one CTA per SM, strided over a virtual item
+// space; items outside the causal triangle are skipped by every role alike.
+//
+// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM owner and
+// MMA issuer, warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4)..).
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace dsa {
+namespace {
+
+constexpr int kBlockK = 128;      // keys per tile (MMA M)
+constexpr int kN = 256;           // MMA N = queries per tile * H_I
+constexpr int kKbPerItem = 16;    // key blocks per work item
+constexpr int kStages = 6;        // key-tile pipeline depth
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
+
+struct Params {
+  const float* q_scale;
+  const float* w;
+  const float* k_scale;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  float* logits;
+  int64_t ld;
+  int B;
+  int n_qg;   // query groups per sequence (virtual)
+  int n_kc;   // key chunks per sequence (virtual)
+  int64_t n_items;
+  DevErr err;
+};
+
+struct Item {
+  int q_row0;   // global query row of the group's first query
+  int k_row0;   // global key row of the sequence's first key
+  int len_q, len_k;
+  int q0;       // local index of the group's first query
+  int nq;       // queries in the group (<= QPT)
+  int kb0;      // first key block (sequence-local, units of kBlockK)
+  int nkb;      // key blocks in the item
+};
+
+template <int QPT>
+__device__ __forceinline__ bool decode_item(int64_t item, const Params& P, Item& it) {
+  const int kc = static_cast<int>(item % P.n_kc);
+  const int64_t rest = item / P.n_kc;
+  const int qg = static_cast<int>(rest % P.n_qg);
+  const int b = static_cast<int>(rest / P.n_qg);
+  if (b >= P.B) return false;
+  const int cq0 = __ldg(P.cu_q + b), cq1 = __ldg(P.cu_q + b + 1);
+  const int ck0 = __ldg(P.cu_k + b), ck1 = __ldg(P.cu_k + b + 1);
+  it.len_q = cq1 - cq0;
+  it.len_k = ck1 - ck0;
+  it.q0 = qg * QPT;
+  if (it.q0 >= it.len_q || it.len_q > it.len_k) return false;
+  it.nq = min(QPT, it.len_q - it.q0);
+  const int p_max = it.len_k - it.len_q + it.q0 + it.nq - 1;
+  const int kbeg = kc * kKbPerItem * kBlockK;
+  const int kend = min(kbeg + kKbPerItem * kBlockK, p_max + 1);
+  if (kbeg >= kend) return false;
+  it.kb0 = kbeg / kBlockK;
+  it.nkb = (kend - kbeg + kBlockK - 1) / kBlockK;
+  it.q_row0 = cq0 + it.q0;
+  it.k_row0 = ck0;
+  return true;
+}
+
+template <int H_I, int D_I>
+struct Layout {
+  static constexpr int QPT = kN / H_I;
+  static constexpr uint32_t kQBytes = kN * D_I;          // one query group tile
+  static constexpr uint32_t kKBytes = kBlockK * D_I;     // one key tile
+  static constexpr uint32_t kOffQ = 0;
+  static constexpr uint32_t kOffK = kOffQ + 2 * kQBytes;
+  static constexpr uint32_t kOffWq = kOffK + kStages * kKBytes;
+  static constexpr uint32_t kOffBar = kOffWq + kN * 4;
+  // barriers: q_full[2], q_empty[2], k_full[S], k_empty[S], acc_full[2], acc_empty[2], drain
+  static constexpr uint32_t kNumBars = 2 + 2 + kStages + kStages + 2 + 2 + 1;
+  static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr uint32_t kBytes = kOffMisc + 16;
+  static constexpr uint32_t kSmem = kBytes + 1024;      // + alignment slack
+  static constexpr uint32_t kSwizzle = D_I == 128 ? kSwizzle128B : kSwizzle64B;
+  static constexpr uint32_t kSbo = 8 * D_I;              // 8 rows of one swizzle width
+  static constexpr uint32_t kIdesc = instr_desc(kFmtE4M3, kFmtE4M3, 0, 0, kBlockK, kN);
+};
+
+template <int H_I, int D_I>
+__global__ void __launch_bounds__(kThreads, 1)
+    indexer_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                   const __grid_constant__ CUtensorMap tmap_k, const Params P) {
+  using L = Layout<H_I, D_I>;
+  constexpr int QPT = L::QPT;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  float* wq_s = reinterpret_cast<float*>(smem + L::kOffWq);
+  const uint32_t bar0 = sbase + L::kOffBar;
+  auto q_full = [&](int i) { return bar0 + 8u * i; };
+  auto q_empty = [&](int i) { return bar0 + 8u * (2 + i); };
+  auto k_full = [&](int i) { return bar0 + 8u * (4 + i); };
+  auto k_empty = [&](int i) { return bar0 + 8u * (4 + kStages + i); };
+  auto acc_full = [&](int i) { return bar0 + 8u * (4 + 2 * kStages + i); };
+  auto acc_empty = [&](int i) { return bar0 + 8u * (6 + 2 * kStages + i); };
+  const uint32_t drain_bar = bar0 + 8u * (8 + 2 * kStages);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(q_full(i), 1);
+      mbar_init(q_empty(i), 1);
+      mbar_init(acc_full(i), 1);
+      mbar_init(acc_empty(i), 1);
+    }
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(k_full(i), 1);
+      mbar_init(k_empty(i), 1);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&tmap_k);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int64_t qc = 0, kc = 0;
+      bool ok = true;
+      for (int64_t item = blockIdx.x; ok && item < P.n_items; item += gridDim.x) {
+        Item it;
+        if (!decode_item<QPT>(item, P, it)) continue;
+        const int qb = static_cast<int>(qc & 1);
+        if (!(ok = mbar_wait(q_empty(qb), static_cast<uint32_t>(((qc >> 1) & 1) ^ 1), P.err))) break;
+        mbar_arrive_expect_tx(q_full(qb), L::kQBytes);
+        tma_load_2d(sbase + L::kOffQ + qb * L::kQBytes, &tmap_q, 0, it.q_row0 * H_I, q_full(qb));
+        ++qc;
+        for (int j = 0; j < it.nkb; ++j) {
+          const int st = static_cast<int>(kc % kStages);
+          const uint32_t par = static_cast<uint32_t>(((kc / kStages) & 1) ^ 1);
+          if (!(ok = mbar_wait(k_empty(st), par, P.err))) break;
+          mbar_arrive_expect_tx(k_full(st), L::kKBytes);
+          tma_load_2d(sbase + L::kOffK + st * L::kKBytes, &tmap_k, 0,
+                      it.k_row0 + (it.kb0 + j) * kBlockK, k_full(st));
+          ++kc;
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        // let this CTA's own loads in flight land before leaving
+        for (int64_t u = (kc > kStages ? kc - kStages : 0); u < kc; ++u)
+          mbar_wait_drain(k_full(static_cast<int>(u % kStages)),
+                          static_cast<uint32_t>((u / kStages) & 1));
+        for (int64_t u = (qc > 2 ? qc - 2 : 0); u < qc; ++u)
+          mbar_wait_drain(q_full(static_cast<int>(u & 1)), static_cast<uint32_t>((u >> 1) & 1));
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int64_t qc = 0, kc = 0, ac = 0;
+      bool ok = true;
+      for (int64_t item = blockIdx.x; ok && item < P.n_items; item += gridDim.x) {
+        Item it;
+        if (!decode_item<QPT>(item, P, it)) continue;
+        const int qb = static_cast<int>(qc & 1);
+        if (!(ok = mbar_wait(q_full(qb), static_cast<uint32_t>((qc >> 1) & 1), P.err))) break;
+        const uint32_t q_addr = sbase + L::kOffQ + qb * L::kQBytes;
+        for (int j = 0; j < it.nkb; ++j) {
+          const int st = static_cast<int>(kc % kStages);
+          if (!(ok = mbar_wait(k_full(st), static_cast<uint32_t>((kc / kStages) & 1), P.err))) break;
+          const int ab = static_cast<int>(ac & 1);
+          if (!(ok = mbar_wait(acc_empty(ab), static_cast<uint32_t>(((ac >> 1) & 1) ^ 1), P.err)))
+            break;
+          tc_fence_after();
+          const uint32_t k_addr = sbase + L::kOffK + st * L::kKBytes;
+          const uint32_t d = tmem + static_cast<uint32_t>(ab) * kN;
+#pragma unroll
+          for (int kk = 0; kk < D_I / 32; ++kk) {
+            const uint64_t adesc = smem_desc(k_addr + kk * 32, 16, L::kSbo, L::kSwizzle);
+            const uint64_t bdesc = smem_desc(q_addr + kk * 32, 16, L::kSbo, L::kSwizzle);
+            mma_f8(d, adesc, bdesc, L::kIdesc, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(k_empty(st));
+          mma_commit(acc_full(ab));
+          ++kc;
+          ++ac;
+        }
+        if (!ok) break;
+        mma_commit(q_empty(qb));
+        ++qc;
+      }
+      // every MMA issued by this thread completes before TMEM is released
+      mma_commit(drain_bar);
+      mbar_wait_drain(drain_bar, 0);
+      if (!ok) *abort_flag = 1;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int et = threadIdx.x - 64;          // 0..127
+    const int sp = warp & 3;                  // TMEM sub-partition of this warp
+    const int row = sp * 32 + lane;           // TMEM lane = key within the tile
+    const uint32_t lane_addr = static_cast<uint32_t>(sp * 32) << 16;
+    int64_t ac = 0;
+    bool ok = true;
+    for (int64_t item = blockIdx.x; ok && item < P.n_items; item += gridDim.x) {
+      Item it;
+      if (!decode_item<QPT>(item, P, it)) continue;
+      // head weights of this query group: wq[qi*H_I + j] = w * q_scale
+      named_bar_sync(1, kEpiThreads);
+      for (int n = et; n < kN; n += kEpiThreads) {
+        const int qi = n / H_I;
+        float v = 0.f;
+        if (qi < it.nq) {
+          const int64_t o = static_cast<int64_t>(it.q_row0 + qi) * H_I + (n % H_I);
+          v = __ldg(P.w + o) * __ldg(P.q_scale + o);
+        }
+        wq_s[n] = v;
+      }
+      named_bar_sync(1, kEpiThreads);
+      for (int j = 0; j < it.nkb; ++j) {
+        const int ab = static_cast<int>(ac & 1);
+        if (et == 0) {
+          if (!mbar_wait(acc_full(ab), static_cast<uint32_t>((ac >> 1) & 1), P.err)) *abort_flag = 1;
+        }
+        named_bar_sync(1, kEpiThreads);
+        if (*abort_flag) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int s_local = (it.kb0 + j) * kBlockK + row;
+        float acc[QPT];
+#pragma unroll
+        for (int qi = 0; qi < QPT; ++qi) acc[qi] = 0.f;
+        const uint32_t dcol = tmem + lane_addr + static_cast<uint32_t>(ab) * kN;
+#pragma unroll
+        for (int ch = 0; ch < kN / 32; ++ch) {
+          if ((ch * 32) / H_I < it.nq) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(dcol + ch * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const int n = ch * 32 + c;
+              acc[n / H_I] = fmaf(wq_s[n], fmaxf(__uint_as_float(v[c]), 0.f), acc[n / H_I]);
+            }
+          }
+        }
+        tc_fence_before();
+        named_bar_sync(1, kEpiThreads);
+        if (et == 0) mbar_arrive(acc_empty(ab));
+        ++ac;
+        if (s_local < it.len_k) {
+          const float ks = __ldg(P.k_scale + it.k_row0 + s_local);
+          const int p0 = it.len_k - it.len_q + it.q0;
+#pragma unroll
+          for (int qi = 0; qi < QPT; ++qi) {
+            if (qi < it.nq && s_local <= p0 + qi)
+              P.logits[static_cast<int64_t>(it.q_row0 + qi) * P.ld + s_local] = acc[qi] * ks;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int H_I, int D_I>
+cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const IndexerArgs& a,
+                     int num_sms, DevErr err, cudaStream_t s) {
+  using L = Layout<H_I, D_I>;
+  Params P;
+  P.q_scale = a.q_scale;
+  P.w = a.w;
+  P.k_scale = a.k_scale;
+  P.cu_q = a.cu_q;
+  P.cu_k = a.cu_k;
+  P.logits = a.logits;
+  P.ld = a.ld;
+  P.B = a.B;
+  P.n_qg = (a.max_len_q + L::QPT - 1) / L::QPT;
+  P.n_kc = (a.max_len_k + kKbPerItem * kBlockK - 1) / (kKbPerItem * kBlockK);
+  P.n_items = static_cast<int64_t>(a.B) * P.n_qg * P.n_kc;
+  P.err = err;
+  if (P.n_items == 0) return cudaSuccess;
+  auto kern = indexer_kernel<H_I, D_I>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(L::kSmem));
+  if (e != cudaSuccess) return e;
+  const int64_t grid = P.n_items < num_sms ? P.n_items : num_sms;
+  kern<<<static_cast<unsigned>(grid), kThreads, L::kSmem, s>>>(tq, tk, P);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_indexer(const CUtensorMap& tq, const CUtensorMap& tk, const IndexerArgs& a,
+                           int num_sms, DevErr err, cudaStream_t s) {
+#define DSA_IDX_CASE(h, d) \
+  if (a.H_I == h && a.d_I == d) return launch_t<h, d>(tq, tk, a, num_sms, err, s);
+  DSA_IDX_CASE(4, 64)
+  DSA_IDX_CASE(8, 64)
+  DSA_IDX_CASE(16, 64)
+  DSA_IDX_CASE(32, 64)
+  DSA_IDX_CASE(64, 64)
+  DSA_IDX_CASE(128, 64)
+  DSA_IDX_CASE(4, 128)
+  DSA_IDX_CASE(8, 128)
+  DSA_IDX_CASE(16, 128)
+  DSA_IDX_CASE(32, 128)
+  DSA_IDX_CASE(64, 128)
+  DSA_IDX_CASE(128, 128)
+#undef DSA_IDX_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace dsa

@@ -1,0 +1,56 @@
+// internal.h -- launchers shared between the C-ABI layer (api.cu) and the
+// kernel translation units.  Not part of the public interface.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ptx.cuh"
+
+namespace dsa {
+
+struct IndexerArgs {
+  const float* q_scale;
+  const float* w;
+  const float* k_scale;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int B, max_len_q, max_len_k;
+  int H_I, d_I;
+  float* logits;
+  int64_t ld;
+};
+
+struct TopkArgs {
+  const float* logits;
+  int64_t ld;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int B, max_len_q, max_len_k;
+  int64_t total_q;
+  int k;
+  int32_t* idx;
+  float* val;
+};
+
+struct MlaArgs {
+  const int32_t* idx;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int B, max_len_q, max_len_k;
+  int64_t total_q, total_k;
+  int H, k;
+  float sm_scale;
+  void* out;
+  float* lse;
+};
+
+// Each returns cudaSuccess or the launch error.
+cudaError_t launch_indexer(const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
+                           const IndexerArgs& a, int num_sms, DevErr err, cudaStream_t s);
+cudaError_t launch_topk(const TopkArgs& a, DevErr err, cudaStream_t s);
+cudaError_t launch_sparse_mla(const CUtensorMap& tmap_q, const CUtensorMap& tmap_kv,
+                              const MlaArgs& a, DevErr err, cudaStream_t s);
+
+}  // namespace dsa

@@ -1,0 +1,422 @@
+// sparse_mla.cu -- sparse attention in the MQA mode of MLA on sm_100a.
+//
+// What it computes ("DeepSeek V3.2 and the lightning indexer", section "How
+// the lightning indexer works": the main attention runs only over the
+// selected entries, and in MQA mode every selected latent serves all query
+// heads; "DeepSeek-V3.2" atlas entry, "Inference efficiency": only the chosen
+// latents of the cache are touched):
+//
+//   out[t,h,:] = sum_{s in S_t} softmax_s(scale * q[t,h,:] . c[s,:]) * c[s,0:512]
+//   lse[t,h]   = log sum_{s in S_t} exp(scale * q[t,h,:] . c[s,:])
+//
+// How (one CTA per (query, group of 64 heads), 192 threads):
+//  * warp 0 (TMA): loads the 64 x 576 bf16 query tile once, then for each
+//    block of 64 selected keys gathers the 576-d latent rows with TMA
+//    tile::gather4 into a 128-byte-swizzled tile (two stages).  The gathered
+//    tile is shared by all 64 heads of the CTA (group-shared selection).
+//  * warp 1 (MMA): S = Q K^T as 36 tcgen05.mma (M=64 heads, N=64 keys, K=16)
+//    into TMEM; after the softmax warps publish P (bf16, in shared memory),
+//    O += P V as 8 tcgen05.mma (M=64, N=256, K=16) with V read MN-major from
+//    the same gathered tile (its first 512 columns).
+//  * warps 2..5 (softmax): read S from TMEM, online softmax in fp32 (exp2,
+//    lazily rescaled maximum), write P, rescale O in TMEM when the maximum
+//    moves, and finally normalise O and store bf16 out and the lse.
+//
+// TMEM (512 columns x 128 lanes): an M=64 accumulator fills lanes 0-15 of
+// each 32-lane sub-partition; a second one at lane offset 16 fills lanes
+// 16-31.  O (64 heads x 512 fp32) takes columns 0..511 at lane offset 0; the
+// two S buffers (64 x 64) take columns 0..63 and 64..127 at lane offset 16.
+// In softmax warp w (sub-partition w%4), threads 16..31 own S rows and
+// threads 0..15 own the O rows of the same heads.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace dsa {
+namespace {
+
+constexpr int kHeads = 64;       // heads per CTA (MMA M)
+constexpr int kBlockN = 64;      // keys per block
+constexpr int kDqk = 576;
+constexpr int kDv = 512;
+constexpr int kChunks = kDqk / 64;                // 9 column chunks of 64
+constexpr uint32_t kChunkBytes = 64 * 128;        // 64 rows x 128 B
+constexpr uint32_t kQBytes = kChunks * kChunkBytes;   // 73728
+constexpr uint32_t kKvBytes = kChunks * kChunkBytes;  // 73728
+constexpr uint32_t kPBytes = kHeads * kBlockN * 2;    // 8192
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffKv = kOffQ + kQBytes;
+constexpr uint32_t kOffP = kOffKv + 2 * kKvBytes;
+constexpr uint32_t kOffBar = kOffP + kPBytes;
+// barriers: q_full, kv_full[2], kv_empty[2], s_full[2], s_free[2], p_full, pv_done, drain
+constexpr uint32_t kNumBars = 12;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+constexpr uint32_t kSmem = kOffMisc + 16 + 1024;
+constexpr int kThreads = 192;
+constexpr int kSmThreads = 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kIdescS = instr_desc(kFmtBF16, kFmtBF16, 0, 0, kHeads, kBlockN);
+constexpr uint32_t kIdescPV = instr_desc(kFmtBF16, kFmtBF16, 0, 1, kHeads, 256);
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+static_assert(kSmem <= 232448, "shared memory budget");
+
+struct Params {
+  const int32_t* idx;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int B, H, k, head_groups;
+  float scale_log2;  // sm_scale * log2(e)
+  __nv_bfloat16* out;
+  float* lse;
+  DevErr err;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    sparse_mla_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                      const __grid_constant__ CUtensorMap tmap_kv, const Params P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + kOffBar;
+  const uint32_t q_full = bar0;
+  auto kv_full = [&](int i) { return bar0 + 8u * (1 + i); };
+  auto kv_empty = [&](int i) { return bar0 + 8u * (3 + i); };
+  auto s_full = [&](int i) { return bar0 + 8u * (5 + i); };
+  auto s_free = [&](int i) { return bar0 + 8u * (7 + i); };
+  const uint32_t p_full = bar0 + 8u * 9;
+  const uint32_t pv_done = bar0 + 8u * 10;
+  const uint32_t drain_bar = bar0 + 8u * 11;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  // ---- which query / heads
+  const int64_t q_row = blockIdx.x / P.head_groups;
+  const int hg = static_cast<int>(blockIdx.x % P.head_groups);
+  int lo = 0, hi = P.B;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(P.cu_q + mid) <= q_row) lo = mid; else hi = mid;
+  }
+  const int b = lo;
+  const int cq0 = __ldg(P.cu_q + b);
+  const int ck0 = __ldg(P.cu_k + b);
+  const int len_q = __ldg(P.cu_q + b + 1) - cq0;
+  const int len_k = __ldg(P.cu_k + b + 1) - ck0;
+  const int p = len_k - len_q + static_cast<int>(q_row - cq0);   // absolute position
+  const int n_sel = min(P.k, p + 1);
+  const int nb = (n_sel + kBlockN - 1) / kBlockN;
+  const int heads_here = min(kHeads, P.H - hg * kHeads);
+  const int32_t* idx_row = P.idx + q_row * P.k;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(kv_full(i), 1);
+      mbar_init(kv_empty(i), 1);
+      mbar_init(s_full(i), 1);
+      mbar_init(s_free(i), 1);
+    }
+    mbar_init(p_full, 1);
+    mbar_init(pv_done, 1);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&tmap_kv);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_o = tmem;                         // + 256*h
+  const uint32_t tmem_s = tmem + (16u << 16);           // + 64*buffer
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, kQBytes);
+      const int32_t y = static_cast<int32_t>(q_row * P.H + hg * kHeads);
+      for (int c = 0; c < kChunks; ++c)
+        tma_load_2d(sbase + kOffQ + c * kChunkBytes, &tmap_q, c * 64, y, q_full);
+    }
+    int j = 0;
+    bool ok = true;
+    for (; j < nb; ++j) {
+      const int st = j & 1;
+      int w_ok = 1;
+      if (lane == 0) w_ok = mbar_wait(kv_empty(st), static_cast<uint32_t>(((j >> 1) & 1) ^ 1), P.err);
+      w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+      if (!w_ok) {
+        ok = false;
+        break;
+      }
+      int32_t rows[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int e = j * kBlockN + (lane & 15) * 4 + q;
+        int s = -1;
+        if (e < n_sel) s = __ldg(idx_row + e);
+        rows[q] = ck0 + ((s >= 0 && s <= p) ? s : 0);
+      }
+      if (lane == 0) mbar_arrive_expect_tx(kv_full(st), kKvBytes);
+      __syncwarp();
+      if (lane < 16) {
+        const uint32_t dst = sbase + kOffKv + st * kKvBytes + lane * 512;
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c)
+          tma_gather4(dst + c * kChunkBytes, &tmap_kv, c * 64, rows[0], rows[1], rows[2], rows[3],
+                      kv_full(st));
+      }
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      mbar_wait_drain(q_full, 0);
+      for (int u = (j > 2 ? j - 2 : 0); u < j; ++u)
+        mbar_wait_drain(kv_full(u & 1), static_cast<uint32_t>((u >> 1) & 1));
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(q_full, 0, P.err);
+      for (int j = 0; ok && j <= nb; ++j) {
+        if (j < nb) {
+          const int st = j & 1;
+          if (!(ok = mbar_wait(kv_full(st), static_cast<uint32_t>((j >> 1) & 1), P.err))) break;
+          if (!(ok = mbar_wait(s_free(st), static_cast<uint32_t>(((j >> 1) & 1) ^ 1), P.err))) break;
+          tc_fence_after();
+          const uint32_t kv = sbase + kOffKv + st * kKvBytes;
+          const uint32_t d = tmem_s + 64u * st;
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = smem_desc(sbase + kOffQ + c * kChunkBytes + kk * 32, 16, 1024,
+                                            kSwizzle128B);
+              const uint64_t bd = smem_desc(kv + c * kChunkBytes + kk * 32, 16, 1024, kSwizzle128B);
+              mma_f16(d, ad, bd, kIdescS, (c | kk) != 0 ? 1u : 0u);
+            }
+          }
+          mma_commit(s_full(st));
+        }
+        if (j >= 1) {
+          const int i = j - 1;
+          const int st = i & 1;
+          if (!(ok = mbar_wait(p_full, static_cast<uint32_t>(i & 1), P.err))) break;
+          tc_fence_after();
+          const uint32_t kv = sbase + kOffKv + st * kKvBytes;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = smem_desc(sbase + kOffP + kk * 32, 16, 1024, kSwizzle128B);
+              const uint64_t bd = smem_desc(kv + (4 * h) * kChunkBytes + kk * 2048, kChunkBytes,
+                                            1024, kSwizzle128B);
+              mma_f16(tmem_o + 256u * h, ad, bd, kIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          mma_commit(kv_empty(st));
+          mma_commit(pv_done);
+        }
+      }
+      mma_commit(drain_bar);
+      mbar_wait_drain(drain_bar, 0);
+      if (!ok) *abort_flag = 1;
+    }
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int et = threadIdx.x - 64;
+    const int sp = warp & 3;
+    const bool is_s = lane >= 16;
+    const int r_s = sp * 16 + (lane - 16);   // S row owned by lanes 16..31
+    const int r_o = sp * 16 + lane;          // O row owned by lanes 0..15
+    const uint32_t lane_base = static_cast<uint32_t>(sp * 32) << 16;
+    float m = -INFINITY;   // running maximum, log2 units
+    float l = 0.f;         // running denominator
+    bool ok = true;
+    uint8_t* p_tile = smem + kOffP;
+    for (int j = 0; j < nb; ++j) {
+      const int st = j & 1;
+      // validity of the 64 entries of this block (each lane checks two)
+      uint32_t vmask_lo, vmask_hi;
+      {
+        const int e0 = j * kBlockN + 2 * lane;
+        const int s0 = e0 < n_sel ? __ldg(idx_row + e0) : -1;
+        const int s1 = e0 + 1 < n_sel ? __ldg(idx_row + e0 + 1) : -1;
+        vmask_lo = __ballot_sync(0xffffffffu, s0 >= 0 && s0 <= p);
+        vmask_hi = __ballot_sync(0xffffffffu, s1 >= 0 && s1 <= p);
+      }
+      if (et == 0 && !mbar_wait(s_full(st), static_cast<uint32_t>((j >> 1) & 1), P.err))
+        *abort_flag = 1;
+      named_bar_sync(1, kSmThreads);
+      if (*abort_flag) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // A 32x32b load covers the warp's whole 32-lane sub-partition, so it
+      // starts at the sub-partition base: lanes 16..31 deliver the S rows.
+      uint32_t v0[32], v1[32];
+      tmem_ld_32x32b_x32(tmem + lane_base + 64u * st, v0);
+      tmem_ld_32x32b_x32(tmem + lane_base + 64u * st + 32, v1);
+      tmem_wait_ld();
+      tc_fence_before();
+      named_bar_sync(1, kSmThreads);
+      if (et == 0) mbar_arrive(s_free(st));
+
+      float x[64];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const uint32_t bits = (c & 1) ? vmask_hi : vmask_lo;
+        const bool valid = (bits >> (c >> 1)) & 1u;
+        const uint32_t raw = c < 32 ? v0[c] : v1[c - 32];
+        x[c] = valid ? __uint_as_float(raw) * P.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, x[c]);
+      }
+      float alpha = 1.f;
+      bool moved = false;
+      if (is_s && mx > m + kRescaleThreshold) {
+        alpha = fast_exp2(m - mx);   // 0 when m = -inf
+        m = mx;
+        moved = true;
+      }
+      // PV of the previous block must be done before P is rewritten and O rescaled
+      if (j >= 1) {
+        if (et == 0 && !mbar_wait(pv_done, static_cast<uint32_t>((j - 1) & 1), P.err))
+          *abort_flag = 1;
+        named_bar_sync(1, kSmThreads);
+        if (*abort_flag) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, moved)) {
+          const float a_lo = __shfl_sync(0xffffffffu, alpha, 16 + (lane >> 2));
+          const float a_hi = __shfl_sync(0xffffffffu, alpha, 24 + (lane >> 2));
+#pragma unroll 1
+          for (int q = 0; q < kDv / 64; ++q) {
+            uint32_t o[32];
+            const uint32_t ta = tmem_o + lane_base + 64u * q;
+            tmem_ld_16x256b_x8(ta, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) {
+              o[4 * rr + 0] = __float_as_uint(__uint_as_float(o[4 * rr + 0]) * a_lo);
+              o[4 * rr + 1] = __float_as_uint(__uint_as_float(o[4 * rr + 1]) * a_lo);
+              o[4 * rr + 2] = __float_as_uint(__uint_as_float(o[4 * rr + 2]) * a_hi);
+              o[4 * rr + 3] = __float_as_uint(__uint_as_float(o[4 * rr + 3]) * a_hi);
+            }
+            tmem_st_16x256b_x8(ta, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      if (is_s) {
+        float sum = 0.f;
+        uint8_t* prow = p_tile + r_s * 128;
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          uint32_t packed[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = c8 * 8 + 2 * e;
+            const float p0 = x[c] == -INFINITY ? 0.f : fast_exp2(x[c] - m);
+            const float p1 = x[c + 1] == -INFINITY ? 0.f : fast_exp2(x[c + 1] - m);
+            sum += p0 + p1;
+            packed[e] = pack_bf16x2(p0, p1);
+          }
+          *reinterpret_cast<uint4*>(prow + ((c8 ^ (r_s & 7)) << 4)) =
+              make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        }
+        l = l * alpha + sum;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(1, kSmThreads);
+      if (et == 0) mbar_arrive(p_full);
+    }
+
+    if (ok) {
+      if (et == 0 && !mbar_wait(pv_done, static_cast<uint32_t>((nb - 1) & 1), P.err))
+        *abort_flag = 1;
+      named_bar_sync(1, kSmThreads);
+      ok = !*abort_flag;
+    }
+    if (ok) {
+      tc_fence_after();
+      const float inv_l_s = l > 0.f ? 1.f / l : 0.f;
+      const float inv_l = __shfl_sync(0xffffffffu, inv_l_s, (lane & 15) + 16);
+      if (is_s && r_s < heads_here && P.lse) {
+        const int h = hg * kHeads + r_s;
+        P.lse[q_row * P.H + h] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      }
+      const int h = hg * kHeads + r_o;
+      __nv_bfloat16* orow = P.out + (q_row * P.H + h) * kDv;
+      const bool store = !is_s && r_o < heads_here;
+#pragma unroll 1
+      for (int cc = 0; cc < kDv / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld_32x32b_x32(tmem_o + lane_base + 32u * cc, o);
+        tmem_wait_ld();
+        if (store) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l,
+                                __uint_as_float(o[2 * e + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * cc);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_sparse_mla(const CUtensorMap& tq, const CUtensorMap& tkv, const MlaArgs& a,
+                              DevErr err, cudaStream_t s) {
+  Params P;
+  P.idx = a.idx;
+  P.cu_q = a.cu_q;
+  P.cu_k = a.cu_k;
+  P.B = a.B;
+  P.H = a.H;
+  P.k = a.k;
+  P.head_groups = (a.H + kHeads - 1) / kHeads;
+  P.scale_log2 = a.sm_scale * 1.4426950408889634f;
+  P.out = reinterpret_cast<__nv_bfloat16*>(a.out);
+  P.lse = a.lse;
+  P.err = err;
+  const int64_t grid = a.total_q * P.head_groups;
+  if (grid == 0) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(sparse_mla_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmem));
+  if (e != cudaSuccess) return e;
+  sparse_mla_kernel<<<static_cast<unsigned>(grid), kThreads, kSmem, s>>>(tq, tkv, P);
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

@@ -25,3 +25,11 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _built_library():
+    """Build libdsa.so (no-op when fresh) so every test runs the real library."""
+    from sparse_attention_08_b200 import _build
+    _build.build()
+    yield

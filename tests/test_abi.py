@@ -1,0 +1,120 @@
+"""The C ABI on the host (no GPU needed): the library loads, exports every
+symbol include/dsa.h declares, and rejects bad arguments with the documented
+status before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_attention_08_b200 as dsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dsa.h")
+
+OK, INVALID, UNSUPPORTED, ALIGN, WORKSPACE, CUDA = 0, 1, 2, 3, 4, 5
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^DSA_API\s+[\w\*\s]+?\b(dsa_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declarations_are_exported():
+    names = _declared()
+    assert names == sorted(dsa.EXPORTED)
+    lib = dsa.load()
+    for n in names:
+        assert hasattr(lib, n), n
+    # nothing but the ABI is exported from the C side
+    assert dsa.dsa_version() == "0.1.0"
+
+
+def test_status_strings():
+    for s in range(8):
+        assert dsa.dsa_status_string(s)
+    assert dsa.dsa_status_string(99) == "unknown status"
+
+
+def test_workspace_size():
+    T, L, k = 1000, 1001, 64
+    ld = 1004
+    expect = (T * ld * 4 + 255) // 256 * 256 + (T * k * 4 + 255) // 256 * 256
+    assert dsa.dsa_forward_workspace_size(T, L, k) == expect
+    assert dsa.dsa_forward_workspace_size(-1, L, k) == 0
+
+
+def _fake(addr=0x10000):
+    return ctypes.c_void_p(addr)
+
+
+def test_indexer_argument_checks_before_device():
+    lib = dsa.load()
+    p = _fake()
+    args = dict(q=p, qs=p, w=p, k=p, ks=p, cq=p, ck=p, B=1, mlq=64, mlk=64, tq=64, tk=64, H_I=64,
+                d_I=128, lg=p, ld=64)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.dsa_indexer_logits(a["q"], a["qs"], a["w"], a["k"], a["ks"], a["cq"], a["ck"],
+                                      a["B"], a["mlq"], a["mlk"], a["tq"], a["tk"], a["H_I"],
+                                      a["d_I"], a["lg"], a["ld"], None)
+    assert call(q=None) == INVALID
+    assert call(cq=None) == INVALID
+    assert call(H_I=48) == UNSUPPORTED
+    assert call(d_I=96) == UNSUPPORTED
+    assert call(ld=32) == INVALID                  # ld < max_len_k
+    assert call(ld=66) == ALIGN                    # row stride not 16-byte
+    assert call(lg=_fake(0x10004)) == ALIGN
+    assert call(mlq=65, mlk=64) == INVALID         # more queries than keys
+    assert call(tq=65) == INVALID                  # total beyond B * max_len
+    assert call(tq=0) == OK                        # nothing to do, no launch
+    if not _have_gpu():
+        assert call() == CUDA                      # no device: fails loudly
+
+
+def test_topk_and_attention_argument_checks():
+    lib = dsa.load()
+    p = _fake()
+    assert lib.dsa_topk(p, 64, p, p, 1, 64, 64, 64, 0, p, None, None) == UNSUPPORTED
+    assert lib.dsa_topk(p, 64, p, p, 1, 64, 64, 64, 5000, p, None, None) == UNSUPPORTED
+    assert lib.dsa_topk(None, 64, p, p, 1, 64, 64, 64, 16, p, None, None) == INVALID
+    assert lib.dsa_topk(p, 64, p, p, 1, 64, 64, 64, 16, _fake(0x10008), None, None) == ALIGN
+    f = ctypes.c_float(1.0 / 24)
+    mla = lib.dsa_sparse_mla_fwd
+    assert mla(p, p, p, p, p, 1, 64, 64, 64, 64, 128, 512, 512, 64, f, p, None, None) == UNSUPPORTED
+    assert mla(p, p, p, p, p, 1, 64, 64, 64, 64, 48, 576, 512, 64, f, p, None, None) == UNSUPPORTED
+    assert mla(p, p, p, p, p, 1, 64, 64, 64, 64, 128, 576, 512, 64, ctypes.c_float(-1.0), p, None,
+               None) == INVALID
+    assert mla(p, None, p, p, p, 1, 64, 64, 64, 64, 128, 576, 512, 64, f, p, None, None) == INVALID
+    assert mla(p, p, p, p, p, 1, 64, 64, 64, 64, 128, 576, 512, 64, f, _fake(0x10002), None,
+               None) == ALIGN
+
+
+def test_forward_workspace_checks():
+    lib = dsa.load()
+    p = _fake()
+    f = ctypes.c_float(1.0 / 24)
+    need = dsa.dsa_forward_workspace_size(64, 64, 16)
+
+    def fwd(ws, nbytes):
+        return lib.dsa_forward(p, p, p, p, p, p, p, p, p, 1, 64, 64, 64, 64, 64, 128, 128, 576, 512,
+                               16, f, p, None, None, ws, nbytes, None)
+    assert fwd(None, need) == WORKSPACE
+    assert fwd(p, need - 1) == WORKSPACE
+    assert fwd(_fake(0x10001), need) == ALIGN
+
+
+def _have_gpu():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+@pytest.mark.gpu
+def test_device_error_word_starts_clear():
+    import torch
+    torch.zeros(1, device="cuda")
+    assert dsa.dsa_get_device_error() == OK

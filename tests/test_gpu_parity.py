@@ -1,0 +1,297 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs.  Small cases are compared element by element over whole
+tensors (several tiles plus ragged tails); the full-size configurations run in
+the launch configuration the benchmark times and are compared on sampled
+query rows, which the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_attention_08_b200 import workloads as W
+from tests import dsa_cases as C
+
+pytestmark = pytest.mark.gpu
+
+
+def _small(**kw):
+    wl = W.make_small(**kw)
+    return wl, wl.to("cuda")
+
+
+def _p_rows(wl, b, rows):
+    q0, q1, k0, k1 = C.seq_slices(wl, b)
+    return [(k1 - k0) - (q1 - q0) + int(i) for i in rows]
+
+
+# --------------------------------------------------------------------------
+# Indexer
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("H_I,d_I", [(4, 64), (64, 128), (16, 128), (8, 64)])
+def test_indexer_integer_inputs_exact(H_I, d_I):
+    cpu, gpu = _small(H_I=H_I, d_I=d_I, H=16, L=333, k=64, integer=True, seed=101)
+    g = C.np_(C.gpu_indexer(gpu))
+    C.assert_no_device_error()
+    o = C.oracle_scores(cpu, 0)
+    rows = np.arange(cpu.T_q)
+    C.check_indexer(g, o, None, _p_rows(cpu, 0, rows), exact=True)
+
+
+@pytest.mark.parametrize("H_I,d_I", [(64, 128), (32, 64)])
+def test_indexer_real_varlen_and_chunk(H_I, d_I):
+    # two sequences: a 700-token prefill and a 150-query chunk at the end of
+    # a 520-token cache (positions 370..519)
+    cpu, gpu = _small(H_I=H_I, d_I=d_I, H=16, lens=[700, 520], lens_q=[700, 150], k=64, seed=102)
+    g = C.np_(C.gpu_indexer(gpu))
+    C.assert_no_device_error()
+    for b in range(2):
+        q0, q1, _, _ = C.seq_slices(cpu, b)
+        rows = np.arange(q1 - q0)
+        o = C.oracle_scores(cpu, b)
+        bound = C.oracle_scores(cpu, b, abs_bound=True)
+        C.check_indexer(g[q0:q1], o, bound, _p_rows(cpu, b, rows))
+        # entries beyond the causal limit stay untouched
+        for r in (0, len(rows) // 2):
+            p = _p_rows(cpu, b, [r])[0]
+            assert np.all(np.isnan(g[q0 + r, p + 1:cpu.max_len_k]))
+
+
+# --------------------------------------------------------------------------
+# Top-k (same fp32 scores on both sides -> bit-exact)
+# --------------------------------------------------------------------------
+
+def _topk_vs_oracle(cpu, gpu, logits_gpu, check_val=True):
+    idx, val = C.gpu_topk(gpu, logits_gpu)
+    C.assert_no_device_error()
+    g_idx, g_val = C.np_(idx), C.np_(val)
+    L = C.np_(logits_gpu).astype(np.float64)
+    for b in range(cpu.B):
+        q0, q1, _, k1k = C.seq_slices(cpu, b)
+        n_q, n_k = q1 - q0, cpu.lens_k[b]
+        sc = np.nan_to_num(L[q0:q1, :n_k], nan=0.0)
+        o_idx = oracle.topk(sc, n_q, cpu.k)
+        assert np.array_equal(g_idx[q0:q1], o_idx), f"seq {b}: top-k differs"
+        if check_val:
+            for r in range(n_q):
+                sel = o_idx[r][o_idx[r] >= 0]
+                assert np.array_equal(g_val[q0 + r, : len(sel)].astype(np.float64), sc[r, sel])
+                assert np.all(np.isnan(g_val[q0 + r, len(sel):]))
+
+
+def test_topk_exact_integer_scores_with_ties():
+    cpu, gpu = _small(H_I=4, d_I=64, H=16, lens=[900, 400], lens_q=[900, 77], k=128, integer=True,
+                      seed=103)
+    _topk_vs_oracle(cpu, gpu, C.gpu_indexer(gpu))
+
+
+def test_topk_exact_real_scores():
+    cpu, gpu = _small(H_I=64, d_I=128, H=16, L=1500, k=256, seed=104)
+    _topk_vs_oracle(cpu, gpu, C.gpu_indexer(gpu))
+
+
+@pytest.mark.parametrize("k", [1, 7, 2048, 4096])
+def test_topk_exact_adversarial_rows(k):
+    # hand-made score rows: constant rows, signed zeros, heavy ties, huge
+    # magnitudes, a long row (50000 > the shared-memory-sized rows)
+    n = 50000
+    lens = [n, 3000, 5000]
+    g = torch.Generator().manual_seed(k)
+    rows = []
+    rows.append(torch.zeros(n))
+    r = torch.randint(-3, 4, (n,), generator=g).float()
+    r[torch.rand(n, generator=g) < 0.3] = -0.0
+    rows.append(r)
+    rows.append(torch.randn(n, generator=g) * 1e30)
+    rows.append(torch.where(torch.rand(n, generator=g) < 0.5, torch.tensor(-1.0),
+                            torch.tensor(1.0)))
+    logits = torch.full((len(rows) + 2, n), float("nan"))
+    for i, rr in enumerate(rows):
+        logits[i] = rr
+    T_q = logits.shape[0]
+    # sequence 0: the 4 hand rows are its last 4 queries of a length-n
+    # sequence; sequences 1 and 2: single decode rows
+    lens_q = [len(rows), 1, 1]
+    logits[len(rows), :3000] = torch.randn(3000, generator=g)
+    logits[len(rows) + 1, :5000] = torch.randint(0, 2, (5000,), generator=g).float()
+    cu_q = torch.tensor([0, len(rows), len(rows) + 1, len(rows) + 2], dtype=torch.int32)
+    cu_k = torch.tensor([0, n, n + 3000, n + 8000], dtype=torch.int32)
+    lg = logits.cuda()
+    idx = torch.full((T_q, k), -7, dtype=torch.int32, device="cuda")
+    val = torch.empty((T_q, k), dtype=torch.float32, device="cuda")
+    from sparse_attention_08_b200 import dsa_topk
+    dsa_topk(lg, cu_q.cuda(), cu_k.cuda(), 3, len(rows), n, k, idx, val)
+    C.assert_no_device_error()
+    gi = C.np_(idx)
+    L = logits.numpy().astype(np.float64)
+    for b in range(3):
+        q0, q1 = int(cu_q[b]), int(cu_q[b + 1])
+        n_k = lens[b]
+        o = oracle.topk(np.nan_to_num(L[q0:q1, :n_k], nan=0.0), q1 - q0, k)
+        assert np.array_equal(gi[q0:q1], o), f"sequence {b}"
+
+
+# --------------------------------------------------------------------------
+# Sparse attention (oracle fed the GPU's indices)
+# --------------------------------------------------------------------------
+
+def _attention_vs_oracle(cpu, gpu, idx_gpu):
+    out, lse = C.gpu_attention(gpu, idx_gpu)
+    C.assert_no_device_error()
+    g_out, g_lse, g_idx = C.np_(out.float()), C.np_(lse), C.np_(idx_gpu)
+    o_all, ol_all, g_all, gl_all = [], [], [], []
+    for b in range(cpu.B):
+        q0, q1, _, _ = C.seq_slices(cpu, b)
+        rows = np.arange(q1 - q0)
+        o, ol = C.oracle_attention(cpu, b, g_idx[q0:q1], rows)
+        o_all.append(o)
+        ol_all.append(ol)
+        g_all.append(g_out[q0:q1])
+        gl_all.append(g_lse[q0:q1])
+    return C.check_attention(np.concatenate(g_all), np.concatenate(o_all),
+                             np.concatenate(gl_all), np.concatenate(ol_all))
+
+
+@pytest.mark.parametrize("H,k", [(16, 64), (128, 100), (64, 256), (32, 130)])
+def test_attention_small(H, k):
+    cpu, gpu = _small(H_I=8, d_I=64, H=H, lens=[400, 300], lens_q=[400, 90], k=k, seed=105)
+    idx, _ = C.gpu_topk(gpu, C.gpu_indexer(gpu), with_val=False)
+    _attention_vs_oracle(cpu, gpu, idx)
+
+
+def test_attention_rescales_when_the_maximum_jumps():
+    # Later keys carry much larger latents, so the running softmax maximum
+    # jumps by far more than the lazy-rescale threshold several times per row.
+    cpu, gpu = _small(H_I=8, d_I=64, H=128, L=700, k=512, seed=106, q_div=2.0)
+    ramp = (1.0 + torch.arange(cpu.T_k, dtype=torch.float32) / 40.0)[:, None]
+    cpu.kv = (cpu.kv.float() * ramp).to(torch.bfloat16)
+    gpu.kv = cpu.kv.cuda()
+    idx, _ = C.gpu_topk(gpu, C.gpu_indexer(gpu), with_val=False)
+    _attention_vs_oracle(cpu, gpu, idx)
+
+
+def test_attention_skips_invalid_entries():
+    cpu, gpu = _small(H_I=8, d_I=64, H=64, L=300, k=128, seed=107)
+    idx, _ = C.gpu_topk(gpu, C.gpu_indexer(gpu), with_val=False)
+    bad = idx.clone()
+    bad[5:, 3] = -1                 # holes inside the valid prefix
+    bad[200:, 10] = 100000          # beyond p: skipped
+    _attention_vs_oracle(cpu, gpu, bad)
+
+
+# --------------------------------------------------------------------------
+# End to end
+# --------------------------------------------------------------------------
+
+def test_forward_end_to_end_small_varlen():
+    cpu, gpu = _small(H_I=64, d_I=128, H=128, lens=[1100, 700, 300], lens_q=[1100, 1, 45], k=256,
+                      seed=108)
+    idx, out, lse = C.gpu_forward(gpu)
+    C.assert_no_device_error()
+    g_idx, g_out, g_lse = C.np_(idx), C.np_(out.float()), C.np_(lse)
+    for b in range(cpu.B):
+        q0, q1, _, _ = C.seq_slices(cpu, b)
+        rows = np.arange(q1 - q0)
+        sc = C.oracle_scores(cpu, b)
+        o_idx = oracle.topk(np.nan_to_num(sc, nan=0.0), q1 - q0, cpu.k)
+        C.check_topk_near_cut(g_idx[q0:q1], o_idx, sc, _p_rows(cpu, b, rows), cpu.k)
+        o, ol = C.oracle_attention(cpu, b, g_idx[q0:q1], rows)
+        C.check_attention(g_out[q0:q1], o, g_lse[q0:q1], ol)
+
+
+def test_config0_full_exact():
+    cpu = W.make_prefill(0)
+    gpu = cpu.to("cuda")
+    logits = C.gpu_indexer(gpu)
+    idx, out, lse = C.gpu_forward(gpu)
+    C.assert_no_device_error()
+    o_sc = C.oracle_scores(cpu, 0)
+    rows = np.arange(cpu.T_q)
+    C.check_indexer(C.np_(logits), o_sc, None, _p_rows(cpu, 0, rows), exact=True)
+    # scores are exact, so the selection must be bit-exact end to end
+    o_idx = oracle.topk(np.nan_to_num(o_sc, nan=0.0), cpu.T_q, cpu.k)
+    assert np.array_equal(C.np_(idx), o_idx)
+    o, ol = C.oracle_attention(cpu, 0, o_idx, rows)
+    C.check_attention(C.np_(out.float()), o, C.np_(lse), ol)
+
+
+# --------------------------------------------------------------------------
+# Full-size configurations, sampled rows
+# --------------------------------------------------------------------------
+
+def _sample_rows(n_q, n_k, k, extra, seed):
+    rng = np.random.default_rng(seed)
+    base = {0, min(n_q - 1, 1), n_q - 1}
+    off = n_k - n_q
+    for p in (k - 2, k - 1, k, k + 1):
+        if 0 <= p - off < n_q:
+            base.add(p - off)
+    base.update(int(x) for x in rng.integers(0, n_q, size=extra))
+    return np.array(sorted(base), dtype=np.int64)
+
+
+def _sampled_parity(wl_gpu, b, rows, idx, out, lse, logits=None):
+    """Oracle on sampled query rows of sequence b, each at its own position
+    (the oracle evaluates exactly those rows of the full problem)."""
+    q0, q1, k0, k1 = C.seq_slices(wl_gpu, b)
+    n_q, n_k = q1 - q0, k1 - k0
+    rows = np.asarray(rows, dtype=np.int64)
+    pos = rows + (n_k - n_q)
+    t = torch.as_tensor(q0 + rows, device=wl_gpu.q8.device)
+    k8 = C.np_(wl_gpu.k8[k0:k1])
+    ks = C.np_(wl_gpu.k_scale[k0:k1])
+    q8, qs, w = C.np_(wl_gpu.q8[t]), C.np_(wl_gpu.q_scale[t]), C.np_(wl_gpu.w[t])
+    sc = oracle.indexer_at(q8, qs, w, k8, ks, pos)
+    if logits is not None:
+        bound = oracle.indexer_at(q8 & 0x7F, qs, np.abs(w), k8 & 0x7F, ks, pos)
+        C.check_indexer(C.np_(logits[t]), sc, bound, list(pos))
+    o_idx = np.stack([oracle.topk(sc[r:r + 1, : p + 1], 1, wl_gpu.k)[0]
+                      for r, p in enumerate(pos)])
+    g_idx = C.np_(idx[t])
+    C.check_topk_near_cut(g_idx, o_idx, sc, list(pos), wl_gpu.k)
+    o, ol = oracle.sparse_mla_at(C.bits(wl_gpu.q[t]), C.bits(wl_gpu.kv[k0:k1]), g_idx, pos,
+                                 wl_gpu.scale)
+    return C.check_attention(C.np_(out[t].float()), o, C.np_(lse[t]), ol)
+
+
+def test_config1_sampled():
+    wl = W.make_prefill(1, device="cuda")
+    logits = C.gpu_indexer(wl)
+    idx, out, lse = C.gpu_forward(wl)
+    C.assert_no_device_error()
+    rows = _sample_rows(wl.T_q, wl.T_k, wl.k, 12, seed=1)
+    _sampled_parity(wl, 0, rows, idx, out, lse, logits=logits)
+
+
+def test_config2_sampled_bench_launch():
+    wl = W.make_prefill(2, device="cuda")
+    idx, out, lse = C.gpu_forward(wl)
+    C.assert_no_device_error()
+    rows = _sample_rows(wl.T_q, wl.T_k, wl.k, 6, seed=2)
+    _sampled_parity(wl, 0, rows, idx, out, lse)
+    # properties that hold at any size, checked on every row
+    g = C.np_(idx)
+    n = np.minimum(np.arange(wl.T_q) + 1, wl.k)
+    assert np.array_equal((g >= 0).sum(axis=1), n)
+    valid = g >= 0
+    assert np.all(np.diff(g, axis=1)[valid[:, 1:]] > 0)
+    assert torch.isfinite(out.float()).all()
+
+
+def test_config3_decode_sampled():
+    wl = W.make_decode(3, device="cuda")
+    idx, out, lse = C.gpu_forward(wl)
+    C.assert_no_device_error()
+    for b in (0, 17, 63):
+        _sampled_parity(wl, b, np.array([0]), idx, out, lse)
+
+
+def test_config4_last_chunk_sampled():
+    full = W.make_prefill(4, device="cuda")
+    C_ = full.cfg.L // full.cfg.chunks
+    wl = W.chunk_of(full, full.cfg.chunks - 1, C_)
+    idx, out, lse = C.gpu_forward(wl)
+    C.assert_no_device_error()
+    rows = _sample_rows(wl.T_q, wl.T_k, wl.k, 3, seed=4)
+    _sampled_parity(wl, 0, rows, idx, out, lse)

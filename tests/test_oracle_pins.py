@@ -320,3 +320,23 @@ def test_golden_sparse_budget():
         L, k = row["L"], row["k"]
         assert k * (k + 1) // 2 + (L - k) * k == row["attended_pairs"]
         assert L * (L + 1) // 2 == row["causal_pairs"]
+
+
+def test_position_explicit_entries_match_row_entries():
+    # the *_at entry points evaluate rows at given positions; on rows of a
+    # whole sequence they must reproduce the row-indexed entry points bitwise
+    wl = W.make_small(H_I=4, d_I=16, H=2, L=60, k=8, seed=32)
+    rows = np.array([0, 7, 31, 59], dtype=np.int64)
+    q8, qs, w = _np(wl.q8), _np(wl.q_scale), _np(wl.w)
+    k8, ks = _np(wl.k8), _np(wl.k_scale)
+    qb, kvb = _bits(wl.q), _bits(wl.kv)
+    sc = oracle.indexer(q8, qs, w, k8, ks, rows=rows)
+    sc_at = oracle.indexer_at(q8[rows], qs[rows], w[rows], k8, ks, rows)
+    assert np.array_equal(np.isnan(sc), np.isnan(sc_at))
+    assert np.array_equal(np.nan_to_num(sc), np.nan_to_num(sc_at))
+    idx, out, lse = oracle.forward(q8, qs, w, k8, ks, qb, kvb, 8, wl.scale, rows=rows)
+    i2, o2, l2 = oracle.forward_at(q8[rows], qs[rows], w[rows], k8, ks, qb[rows], kvb, rows, 8,
+                                   wl.scale)
+    assert np.array_equal(idx, i2) and np.array_equal(out, o2) and np.array_equal(lse, l2)
+    o3, l3 = oracle.sparse_mla_at(qb[rows], kvb, idx, rows, wl.scale)
+    assert np.array_equal(out, o3) and np.array_equal(lse, l3)
