@@ -66,6 +66,28 @@ def dist_env():
     return world, rank, local
 
 
+def rank_seed(cfg_id, rank):
+    """Each rank runs its own sequence: rank 0 uses the workload's seed."""
+    from sparse_attention_08_b200 import workloads as W
+    return W.seed_of(cfg_id) + 1000 * rank
+
+
+def max_over_ranks(x: float) -> float:
+    """Maximum of a per-rank float over the process group (identity alone)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(world: int, queries_per_rank: int, step_ms: float) -> float:
+    """Whole-job query-tokens/s: every rank's queries over the slowest rank's step."""
+    return world * queries_per_rank / (step_ms / 1e3)
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -212,7 +234,7 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     dsa.load()
     cfg = W.CONFIGS[args.config]
-    seed = W.seed_of(args.config) + 1000 * rank
+    seed = rank_seed(args.config, rank)
     wl = W.make_prefill(args.config, device="cuda", seed=seed)
     H_I, d_I, H = wl.q8.shape[1], wl.q8.shape[2], wl.q.shape[1]
     ld = (wl.max_len_k + 3) // 4 * 4
@@ -268,12 +290,8 @@ def run_ours(args):
                    for i in range(args.steps)])             # ms per stage per step
     step_ms = float(st.sum(axis=1).mean())
     stage_ms = st.mean(axis=0)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([step_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms = float(t.item())
-    value = world * wl.T_q / (step_ms / 1e3)
+    step_ms = max_over_ranks(step_ms)
+    value = aggregate_value(world, wl.T_q, step_ms)
 
     # ---- roofline of the dominant kernel and of the whole step
     peaks = measured_peaks()
@@ -370,13 +388,8 @@ def run_e2e(dsa, wl, args, world, local, stream):
     for i in range(args.e2e_steps):
         one(evs[i])
     torch.cuda.synchronize()
-    ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": round(world * wl.T_q / (ms / 1e3), 1), "unit": UNIT,
+    ms = max_over_ranks(float(np.mean([e[0].elapsed_time(e[1]) for e in evs])))
+    return {"value": round(aggregate_value(world, wl.T_q, ms), 1), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": round(ms, 3), "steps": args.e2e_steps, "api": "dsa_forward"}
 

@@ -243,7 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r_o = sp * 16 + lane;          // O row owned by lanes 0..15
     const uint32_t lane_base = static_cast<uint32_t>(sp * 32) << 16;
     float m = -INFINITY;   // running maximum, log2 units
-    float l = 0.f;         // running denominator
+    float l = 0.f;         // running denominator (fp32 probabilities), for the lse
+    float lr = 0.f;        // running denominator of the bf16 P the MMA consumes, for O
     bool ok = true;
     uint8_t* p_tile = smem + kOffP;
     for (int j = 0; j < nb; ++j) {
@@ -324,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (is_s) {
-        float sum = 0.f;
+        float sum = 0.f, sum_r = 0.f;
         uint8_t* prow = p_tile + r_s * 128;
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
@@ -336,11 +337,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float p1 = x[c + 1] == -INFINITY ? 0.f : fast_exp2(x[c + 1] - m);
             sum += p0 + p1;
             packed[e] = pack_bf16x2(p0, p1);
+            // the weights O receives are the rounded ones: normalise by their sum
+            sum_r += __uint_as_float(packed[e] << 16) + __uint_as_float(packed[e] & 0xFFFF0000u);
           }
           *reinterpret_cast<uint4*>(prow + ((c8 ^ (r_s & 7)) << 4)) =
               make_uint4(packed[0], packed[1], packed[2], packed[3]);
         }
         l = l * alpha + sum;
+        lr = lr * alpha + sum_r;
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -356,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) {
       tc_fence_after();
-      const float inv_l_s = l > 0.f ? 1.f / l : 0.f;
+      const float inv_l_s = lr > 0.f ? 1.f / lr : 0.f;
       const float inv_l = __shfl_sync(0xffffffffu, inv_l_s, (lane & 15) + 16);
       if (is_s && r_s < heads_here && P.lse) {
         const int h = hg * kHeads + r_s;

@@ -161,11 +161,15 @@ def test_attention_small(H, k):
 
 
 def test_attention_rescales_when_the_maximum_jumps():
-    # Later keys carry much larger latents, so the running softmax maximum
-    # jumps by far more than the lazy-rescale threshold several times per row.
-    cpu, gpu = _small(H_I=8, d_I=64, H=128, L=700, k=512, seed=106, q_div=2.0)
+    # The RoPE dims (512..575) of later keys are scaled up, so the logits grow
+    # along the key index and the running softmax maximum jumps by far more
+    # than the lazy-rescale threshold several times per row, while the value
+    # dims keep the workload's N(0,1) scale.
+    cpu, gpu = _small(H_I=8, d_I=64, H=128, L=700, k=512, seed=106, q_div=0.5)
     ramp = (1.0 + torch.arange(cpu.T_k, dtype=torch.float32) / 40.0)[:, None]
-    cpu.kv = (cpu.kv.float() * ramp).to(torch.bfloat16)
+    kv = cpu.kv.float()
+    kv[:, 512:] *= ramp
+    cpu.kv = kv.to(torch.bfloat16)
     gpu.kv = cpu.kv.cuda()
     idx, _ = C.gpu_topk(gpu, C.gpu_indexer(gpu), with_val=False)
     _attention_vs_oracle(cpu, gpu, idx)
