@@ -9,25 +9,27 @@
 //   out[t,h,:] = sum_{s in S_t} softmax_s(scale * q[t,h,:] . c[s,:]) * c[s,0:512]
 //   lse[t,h]   = log sum_{s in S_t} exp(scale * q[t,h,:] . c[s,:])
 //
-// How (one CTA per (query, group of 64 heads), 192 threads):
-//  * warp 0 (TMA): loads the 64 x 576 bf16 query tile once, then for each
-//    block of 64 selected keys gathers the 576-d latent rows with TMA
-//    tile::gather4 into a 128-byte-swizzled tile (two stages).  The gathered
+// How (one CTA per (query, group of 64 heads), 416 threads):
+//  * warps 5..12 (gather): for each block of 64 selected keys, 256 threads
+//    copy the 576-d latent rows with 16-byte cp.async into a 128-byte-swizzled
+//    72 KB tile (two stages).  Eight threads cover one 128-byte row segment,
+//    so every warp instruction moves four full 128-byte lines.  The gathered
 //    tile is shared by all 64 heads of the CTA (group-shared selection).
-//  * warp 1 (MMA): S = Q K^T as 36 tcgen05.mma (M=64 heads, N=64 keys, K=16)
-//    into TMEM; after the softmax warps publish P (bf16, in shared memory),
-//    O += P V as 8 tcgen05.mma (M=64, N=256, K=16) with V read MN-major from
-//    the same gathered tile (its first 512 columns).
-//  * warps 2..5 (softmax): read S from TMEM, online softmax in fp32 (exp2,
-//    lazily rescaled maximum), write P, rescale O in TMEM when the maximum
-//    moves, and finally normalise O and store bf16 out and the lse.
+//  * warp 4 (MMA): loads the 64 x 576 query tile once with TMA, then issues,
+//    whichever is ready first, S = Q K^T (36 tcgen05.mma, M=64 heads, N=64
+//    keys, K=16) into TMEM, or O += P V (8 tcgen05.mma, M=64, N=256, K=16)
+//    with V read MN-major from the first 512 columns of the same tile.
+//  * warps 0..3 (softmax): read S from TMEM, online softmax in fp32 (exp2,
+//    lazily rescaled maximum), write P (bf16) to shared memory, rescale O in
+//    TMEM when the maximum moves, and finally normalise O and store bf16 out
+//    and the lse.
 //
 // TMEM (512 columns x 128 lanes): an M=64 accumulator fills lanes 0-15 of
 // each 32-lane sub-partition; a second one at lane offset 16 fills lanes
 // 16-31.  O (64 heads x 512 fp32) takes columns 0..511 at lane offset 0; the
 // two S buffers (64 x 64) take columns 0..63 and 64..127 at lane offset 16.
-// In softmax warp w (sub-partition w%4), threads 16..31 own S rows and
-// threads 0..15 own the O rows of the same heads.
+// In softmax warp w (sub-partition w), threads 16..31 own S rows and threads
+// 0..15 own the O rows of the same heads.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -55,8 +57,15 @@ constexpr uint32_t kOffBar = kOffP + kPBytes;
 constexpr uint32_t kNumBars = 12;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmem = kOffMisc + 16 + 1024;
-constexpr int kThreads = 192;
-constexpr int kSmThreads = 128;
+
+constexpr int kSmWarps = 4;                 // warps 0..3
+constexpr int kMmaWarp = 4;                 // warp 4
+constexpr int kProdWarp0 = 5;               // warps 5..12
+constexpr int kProdWarps = 8;
+constexpr int kSmThreads = 32 * kSmWarps;
+constexpr int kProdThreads = 32 * kProdWarps;
+constexpr int kThreads = 32 * (kSmWarps + 1 + kProdWarps);   // 416
+constexpr uint32_t kBarSoftmax = 1, kBarProducer = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kIdescS = instr_desc(kFmtBF16, kFmtBF16, 0, 0, kHeads, kBlockN);
 constexpr uint32_t kIdescPV = instr_desc(kFmtBF16, kFmtBF16, 0, 1, kHeads, 256);
@@ -65,6 +74,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 static_assert(kSmem <= 232448, "shared memory budget");
 
 struct Params {
+  const __nv_bfloat16* kv;
   const int32_t* idx;
   const int32_t* cu_q;
   const int32_t* cu_k;
@@ -76,8 +86,7 @@ struct Params {
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
-    sparse_mla_kernel(const __grid_constant__ CUtensorMap tmap_q,
-                      const __grid_constant__ CUtensorMap tmap_kv, const Params P) {
+    sparse_mla_kernel(const __grid_constant__ CUtensorMap tmap_q, const Params P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -93,6 +102,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t drain_bar = bar0 + 8u * 11;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  volatile int* prod_abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -119,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(kv_full(i), 1);
+      mbar_init(kv_full(i), kProdThreads);
       mbar_init(kv_empty(i), 1);
       mbar_init(s_full(i), 1);
       mbar_init(s_free(i), 1);
@@ -128,11 +138,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(pv_done, 1);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
+    *prod_abort = 0;
     fence_barrier_init();
-    tma_prefetch_desc(&tmap_q);
-    tma_prefetch_desc(&tmap_kv);
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), kTmemCols);
     tmem_relinquish();
   }
@@ -141,79 +150,64 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tmem_o = tmem;                         // + 256*h
-  const uint32_t tmem_s = tmem + (16u << 16);           // + 64*buffer
+  const uint32_t tmem_s = tmem + (16u << 16);           // + 64*buffer (MMA destination)
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp >= kProdWarp0) {
+    // ------------------------------------------------------------ latent gather
+    const int tp = threadIdx.x - 32 * kProdWarp0;        // 0..255
+    const int rsub = tp >> 3;                            // rows rsub and rsub + 32
+    const int l8 = tp & 7;                               // 16-byte piece within 128 B
+    const __nv_bfloat16* kv_seq = P.kv + static_cast<int64_t>(ck0) * kDqk;
+    auto load_idx = [&](int j, int r) -> int {
+      const int e = j * kBlockN + r;
+      int s = -1;
+      if (e < n_sel) s = __ldg(idx_row + e);
+      return (s >= 0 && s <= p) ? s : 0;                 // invalid entries read row 0 (masked)
+    };
+    int s0 = nb > 0 ? load_idx(0, rsub) : 0;
+    int s1 = nb > 0 ? load_idx(0, rsub + 32) : 0;
+    for (int j = 0; j < nb; ++j) {
+      const int st = j & 1;
+      const int n0 = j + 1 < nb ? load_idx(j + 1, rsub) : 0;       // prefetch next block
+      const int n1 = j + 1 < nb ? load_idx(j + 1, rsub + 32) : 0;
+      if (tp == 0 &&
+          !mbar_wait(kv_empty(st), static_cast<uint32_t>(((j >> 1) & 1) ^ 1), P.err))
+        *prod_abort = 1;
+      named_bar_sync(kBarProducer, kProdThreads);
+      if (*prod_abort) break;
+      const uint32_t stage = sbase + kOffKv + st * kKvBytes;
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        const int r = rsub + 32 * pass;
+        const __nv_bfloat16* src = kv_seq + static_cast<int64_t>(pass ? s1 : s0) * kDqk + l8 * 8;
+        const uint32_t dst = stage + r * 128 + ((l8 ^ (r & 7)) << 4);
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) cp_async16(dst + c * kChunkBytes, src + c * 64);
+      }
+      cp_async_commit();
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      mbar_arrive(kv_full(st));
+      s0 = n0;
+      s1 = n1;
+    }
+    if (*prod_abort && tp == 0) *abort_flag = 1;
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      tma_prefetch_desc(&tmap_q);
       mbar_arrive_expect_tx(q_full, kQBytes);
       const int32_t y = static_cast<int32_t>(q_row * P.H + hg * kHeads);
       for (int c = 0; c < kChunks; ++c)
         tma_load_2d(sbase + kOffQ + c * kChunkBytes, &tmap_q, c * 64, y, q_full);
-    }
-    int j = 0;
-    bool ok = true;
-    for (; j < nb; ++j) {
-      const int st = j & 1;
-      int w_ok = 1;
-      if (lane == 0) w_ok = mbar_wait(kv_empty(st), static_cast<uint32_t>(((j >> 1) & 1) ^ 1), P.err);
-      w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
-      if (!w_ok) {
-        ok = false;
-        break;
-      }
-      int32_t rows[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int e = j * kBlockN + (lane & 15) * 4 + q;
-        int s = -1;
-        if (e < n_sel) s = __ldg(idx_row + e);
-        rows[q] = ck0 + ((s >= 0 && s <= p) ? s : 0);
-      }
-      if (lane == 0) mbar_arrive_expect_tx(kv_full(st), kKvBytes);
-      __syncwarp();
-      if (lane < 16) {
-        const uint32_t dst = sbase + kOffKv + st * kKvBytes + lane * 512;
-#pragma unroll
-        for (int c = 0; c < kChunks; ++c)
-          tma_gather4(dst + c * kChunkBytes, &tmap_kv, c * 64, rows[0], rows[1], rows[2], rows[3],
-                      kv_full(st));
-      }
-    }
-    if (!ok && lane == 0) {
-      *abort_flag = 1;
-      mbar_wait_drain(q_full, 0);
-      for (int u = (j > 2 ? j - 2 : 0); u < j; ++u)
-        mbar_wait_drain(kv_full(u & 1), static_cast<uint32_t>((u >> 1) & 1));
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
       bool ok = mbar_wait(q_full, 0, P.err);
-      for (int j = 0; ok && j <= nb; ++j) {
-        if (j < nb) {
-          const int st = j & 1;
-          if (!(ok = mbar_wait(kv_full(st), static_cast<uint32_t>((j >> 1) & 1), P.err))) break;
-          if (!(ok = mbar_wait(s_free(st), static_cast<uint32_t>(((j >> 1) & 1) ^ 1), P.err))) break;
-          tc_fence_after();
-          const uint32_t kv = sbase + kOffKv + st * kKvBytes;
-          const uint32_t d = tmem_s + 64u * st;
-#pragma unroll
-          for (int c = 0; c < kChunks; ++c) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = smem_desc(sbase + kOffQ + c * kChunkBytes + kk * 32, 16, 1024,
-                                            kSwizzle128B);
-              const uint64_t bd = smem_desc(kv + c * kChunkBytes + kk * 32, 16, 1024, kSwizzle128B);
-              mma_f16(d, ad, bd, kIdescS, (c | kk) != 0 ? 1u : 0u);
-            }
-          }
-          mma_commit(s_full(st));
-        }
-        if (j >= 1) {
-          const int i = j - 1;
-          const int st = i & 1;
-          if (!(ok = mbar_wait(p_full, static_cast<uint32_t>(i & 1), P.err))) break;
+      int js = 0, jp = 0;          // next block for S, next block for PV
+      uint64_t t_idle = 0;
+      uint32_t spins = 0;
+      while (ok && jp < nb) {
+        bool progress = false;
+        if (jp < js && mbar_try_wait(p_full, static_cast<uint32_t>(jp & 1))) {
+          const int st = jp & 1;
           tc_fence_after();
           const uint32_t kv = sbase + kOffKv + st * kKvBytes;
 #pragma unroll
@@ -223,21 +217,66 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint64_t ad = smem_desc(sbase + kOffP + kk * 32, 16, 1024, kSwizzle128B);
               const uint64_t bd = smem_desc(kv + (4 * h) * kChunkBytes + kk * 2048, kChunkBytes,
                                             1024, kSwizzle128B);
-              mma_f16(tmem_o + 256u * h, ad, bd, kIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
+              mma_f16(tmem_o + 256u * h, ad, bd, kIdescPV, (jp > 0 || kk > 0) ? 1u : 0u);
             }
           }
           mma_commit(kv_empty(st));
           mma_commit(pv_done);
+          ++jp;
+          progress = true;
+        }
+        if (js < nb) {
+          const int st = js & 1;
+          const uint32_t ph = static_cast<uint32_t>((js >> 1) & 1);
+          if (mbar_try_wait(kv_full(st), ph) && mbar_try_wait(s_free(st), ph ^ 1u)) {
+            tc_fence_after();
+            const uint32_t kv = sbase + kOffKv + st * kKvBytes;
+            const uint32_t d = tmem_s + 64u * st;
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = smem_desc(sbase + kOffQ + c * kChunkBytes + kk * 32, 16, 1024,
+                                              kSwizzle128B);
+                const uint64_t bd =
+                    smem_desc(kv + c * kChunkBytes + kk * 32, 16, 1024, kSwizzle128B);
+                mma_f16(d, ad, bd, kIdescS, (c | kk) != 0 ? 1u : 0u);
+              }
+            }
+            mma_commit(s_full(st));
+            ++js;
+            progress = true;
+          }
+        }
+        if (progress) {
+          spins = 0;
+          t_idle = 0;
+        } else if ((++spins & 255u) == 0) {
+          if (launch_failed(P.err)) {
+            ok = false;
+          } else {
+            const uint64_t now = globaltimer_ns();
+            if (t_idle == 0) {
+              t_idle = now;
+            } else if (now - t_idle > kWaitLimitNs) {
+              raise_error(P.err, kErrTimeout);
+              ok = false;
+            }
+          }
         }
       }
+      // every MMA issued by this thread completes before TMEM is released
       mma_commit(drain_bar);
       mbar_wait_drain(drain_bar, 0);
-      if (!ok) *abort_flag = 1;
+      if (!ok) {
+        *abort_flag = 1;
+        mbar_wait_drain(q_full, 0);
+      }
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const int et = threadIdx.x - 64;
-    const int sp = warp & 3;
+    const int et = threadIdx.x;              // 0..127
+    const int sp = warp;                     // sub-partition
     const bool is_s = lane >= 16;
     const int r_s = sp * 16 + (lane - 16);   // S row owned by lanes 16..31
     const int r_o = sp * 16 + lane;          // O row owned by lanes 0..15
@@ -260,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (et == 0 && !mbar_wait(s_full(st), static_cast<uint32_t>((j >> 1) & 1), P.err))
         *abort_flag = 1;
-      named_bar_sync(1, kSmThreads);
+      named_bar_sync(kBarSoftmax, kSmThreads);
       if (*abort_flag) {
         ok = false;
         break;
@@ -268,23 +307,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       // A 32x32b load covers the warp's whole 32-lane sub-partition, so it
       // starts at the sub-partition base: lanes 16..31 deliver the S rows.
-      uint32_t v0[32], v1[32];
-      tmem_ld_32x32b_x32(tmem + lane_base + 64u * st, v0);
-      tmem_ld_32x32b_x32(tmem + lane_base + 64u * st + 32, v1);
+      uint32_t v[64];
+      tmem_ld_32x32b_x64(tmem + lane_base + 64u * st, v);
       tmem_wait_ld();
       tc_fence_before();
-      named_bar_sync(1, kSmThreads);
+      named_bar_sync(kBarSoftmax, kSmThreads);
       if (et == 0) mbar_arrive(s_free(st));
 
-      float x[64];
       float mx = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
         const uint32_t bits = (c & 1) ? vmask_hi : vmask_lo;
         const bool valid = (bits >> (c >> 1)) & 1u;
-        const uint32_t raw = c < 32 ? v0[c] : v1[c - 32];
-        x[c] = valid ? __uint_as_float(raw) * P.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, x[c]);
+        const float x = valid ? __uint_as_float(v[c]) * P.scale_log2 : -INFINITY;
+        v[c] = __float_as_uint(x);
+        mx = fmaxf(mx, x);
       }
       float alpha = 1.f;
       bool moved = false;
@@ -297,32 +334,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (j >= 1) {
         if (et == 0 && !mbar_wait(pv_done, static_cast<uint32_t>((j - 1) & 1), P.err))
           *abort_flag = 1;
-        named_bar_sync(1, kSmThreads);
+        named_bar_sync(kBarSoftmax, kSmThreads);
         if (*abort_flag) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, moved)) {
-          const float a_lo = __shfl_sync(0xffffffffu, alpha, 16 + (lane >> 2));
-          const float a_hi = __shfl_sync(0xffffffffu, alpha, 24 + (lane >> 2));
-#pragma unroll 1
-          for (int q = 0; q < kDv / 64; ++q) {
-            uint32_t o[32];
-            const uint32_t ta = tmem_o + lane_base + 64u * q;
-            tmem_ld_16x256b_x8(ta, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int rr = 0; rr < 8; ++rr) {
-              o[4 * rr + 0] = __float_as_uint(__uint_as_float(o[4 * rr + 0]) * a_lo);
-              o[4 * rr + 1] = __float_as_uint(__uint_as_float(o[4 * rr + 1]) * a_lo);
-              o[4 * rr + 2] = __float_as_uint(__uint_as_float(o[4 * rr + 2]) * a_hi);
-              o[4 * rr + 3] = __float_as_uint(__uint_as_float(o[4 * rr + 3]) * a_hi);
-            }
-            tmem_st_16x256b_x8(ta, o);
-          }
-          tmem_wait_st();
-        }
       }
       if (is_s) {
         float sum = 0.f, sum_r = 0.f;
@@ -333,8 +350,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = c8 * 8 + 2 * e;
-            const float p0 = x[c] == -INFINITY ? 0.f : fast_exp2(x[c] - m);
-            const float p1 = x[c + 1] == -INFINITY ? 0.f : fast_exp2(x[c + 1] - m);
+            const float x0 = __uint_as_float(v[c]), x1 = __uint_as_float(v[c + 1]);
+            const float p0 = x0 == -INFINITY ? 0.f : fast_exp2(x0 - m);
+            const float p1 = x1 == -INFINITY ? 0.f : fast_exp2(x1 - m);
             sum += p0 + p1;
             packed[e] = pack_bf16x2(p0, p1);
             // the weights O receives are the rounded ones: normalise by their sum
@@ -346,16 +364,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         l = l * alpha + sum;
         lr = lr * alpha + sum_r;
       }
+      // rescale O (stable: PV(j-1) has completed, PV(j) waits for p_full)
+      if (j >= 1 && __any_sync(0xffffffffu, moved)) {
+        const float a_lo = __shfl_sync(0xffffffffu, alpha, 16 + (lane >> 2));
+        const float a_hi = __shfl_sync(0xffffffffu, alpha, 24 + (lane >> 2));
+#pragma unroll 1
+        for (int q = 0; q < kDv / 64; ++q) {
+          uint32_t o[32];
+          const uint32_t ta = tmem_o + lane_base + 64u * q;
+          tmem_ld_16x256b_x8(ta, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int rr = 0; rr < 8; ++rr) {
+            o[4 * rr + 0] = __float_as_uint(__uint_as_float(o[4 * rr + 0]) * a_lo);
+            o[4 * rr + 1] = __float_as_uint(__uint_as_float(o[4 * rr + 1]) * a_lo);
+            o[4 * rr + 2] = __float_as_uint(__uint_as_float(o[4 * rr + 2]) * a_hi);
+            o[4 * rr + 3] = __float_as_uint(__uint_as_float(o[4 * rr + 3]) * a_hi);
+          }
+          tmem_st_16x256b_x8(ta, o);
+        }
+        tmem_wait_st();
+      }
       fence_proxy_async_smem();
       tc_fence_before();
-      named_bar_sync(1, kSmThreads);
+      named_bar_sync(kBarSoftmax, kSmThreads);
       if (et == 0) mbar_arrive(p_full);
     }
 
     if (ok) {
       if (et == 0 && !mbar_wait(pv_done, static_cast<uint32_t>((nb - 1) & 1), P.err))
         *abort_flag = 1;
-      named_bar_sync(1, kSmThreads);
+      named_bar_sync(kBarSoftmax, kSmThreads);
       ok = !*abort_flag;
     }
     if (ok) {
@@ -391,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -399,9 +438,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_sparse_mla(const CUtensorMap& tq, const CUtensorMap& tkv, const MlaArgs& a,
-                              DevErr err, cudaStream_t s) {
+cudaError_t launch_sparse_mla(const CUtensorMap& tq, const void* kv, const MlaArgs& a, DevErr err,
+                              cudaStream_t s) {
   Params P;
+  P.kv = static_cast<const __nv_bfloat16*>(kv);
   P.idx = a.idx;
   P.cu_q = a.cu_q;
   P.cu_k = a.cu_k;
@@ -419,7 +459,7 @@ cudaError_t launch_sparse_mla(const CUtensorMap& tq, const CUtensorMap& tkv, con
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmem));
   if (e != cudaSuccess) return e;
-  sparse_mla_kernel<<<static_cast<unsigned>(grid), kThreads, kSmem, s>>>(tq, tkv, P);
+  sparse_mla_kernel<<<static_cast<unsigned>(grid), kThreads, kSmem, s>>>(tq, P);
   return cudaGetLastError();
 }
 
