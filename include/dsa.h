@@ -160,6 +160,37 @@ DSA_API dsa_status_t dsa_forward(const void* q_fp8, const float* q_scale, const 
                          float* lse, int32_t* idx_out, void* workspace, size_t workspace_bytes,
                          void* stream);
 
+/*
+ * dsa_forward for callers that cannot allocate device memory.  The pages have
+ * no counterpart to this call; it exists for users of this library.
+ *
+ * Some callers can't call cudaMalloc: a serving engine that reserves the whole
+ * device for its own pool up front, or a latency-critical loop that cannot take
+ * the device synchronisation an allocation brings.  They pass inputs and
+ * outputs as for dsa_forward but no workspace: the scores and indices live in
+ * one fixed device array of 48 MiB per GPU inside the library (held from when
+ * the library's device code loads on that GPU until the process exits).
+ *
+ *  - Returns DSA_ERR_WORKSPACE, without launching anything, when
+ *    dsa_forward_workspace_size(total_q, max_len_k, k) exceeds 48 MiB
+ *    (e.g. 64 decode queries over 131072-token caches with k = 2048 fit;
+ *    a 32768-token prefill does not).
+ *  - The first call on a device looks up the array's device address with that
+ *    device current; make that first call before any stream capture.
+ *  - All calls share the array and leave their data in it; nothing in it
+ *    needs to start at zero.  Calls that overlap on the GPU (e.g. on two
+ *    streams at once) race on it and must be serialised by the caller.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * Other arguments, results and errors are those of dsa_forward.
+ */
+DSA_API dsa_status_t dsa_forward_noalloc(const void* q_fp8, const float* q_scale, const float* w,
+                                         const void* k_fp8, const float* k_scale, const void* q,
+                                         const void* kv, const int32_t* cu_seqlens_q,
+                                         const int32_t* cu_seqlens_k, int B, int max_len_q,
+                                         int max_len_k, int64_t total_q, int64_t total_k, int H_I,
+                                         int d_I, int H, int d_qk, int d_v, int k, float sm_scale,
+                                         void* out, float* lse, int32_t* idx_out, void* stream);
+
 /* Bytes of workspace dsa_forward needs: an f32 score matrix [total_q,
  * round_up(max_len_k, 4)] plus an int32 index matrix [total_q, k], each
  * 256-byte aligned.  Returns 0 for invalid sizes. */

@@ -14,7 +14,7 @@ import os
 __all__ = [
     "DSAError", "lib_path", "load", "dsa_version", "dsa_status_string",
     "dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward",
-    "dsa_forward_workspace_size", "dsa_get_device_error", "EXPORTED",
+    "dsa_forward_workspace_size", "dsa_get_device_error", "dsa_forward_noalloc", "EXPORTED",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -25,6 +25,7 @@ _lib = None
 EXPORTED = (
     "dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward",
     "dsa_forward_workspace_size", "dsa_status_string", "dsa_get_device_error", "dsa_version",
+    "dsa_forward_noalloc",
 )
 
 STATUS = {
@@ -59,7 +60,10 @@ def load():
     lib.dsa_sparse_mla_fwd.argtypes = [P, P, P, P, P, I, I, I, I64, I64, I, I, I, I, F, P, P, P]
     lib.dsa_forward.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I64, I64, I, I, I, I, I, I, F,
                                 P, P, P, P, ctypes.c_size_t, P]
-    for name in ("dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward"):
+    lib.dsa_forward_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I64, I64, I, I, I, I,
+                                        I, I, F, P, P, P, P]
+    for name in ("dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward",
+                 "dsa_forward_noalloc"):
         getattr(lib, name).restype = I
     lib.dsa_forward_workspace_size.argtypes = [I64, I, I]
     lib.dsa_forward_workspace_size.restype = ctypes.c_size_t
@@ -197,6 +201,33 @@ def dsa_forward(q_fp8, q_scale, w, k_fp8, k_scale, q, kv, cu_seqlens_q, cu_seqle
                             _ptr(workspace), int(workspace.numel() * workspace.element_size()),
                             _stream(stream))
     _check(rc, "dsa_forward")
+
+
+def dsa_forward_noalloc(q_fp8, q_scale, w, k_fp8, k_scale, q, kv, cu_seqlens_q, cu_seqlens_k, B,
+                        max_len_q, max_len_k, k, sm_scale, out, lse, idx_out=None, stream=None):
+    """dsa_forward without a workspace, for callers that cannot allocate device
+    memory: the scratch lives in a fixed 48 MiB device array inside the
+    library (see include/dsa.h).  Raises DSAError(DSA_ERR_WORKSPACE) when the
+    problem's scratch exceeds it."""
+    import torch
+    q8 = q_fp8.view(torch.uint8) if q_fp8.dtype == torch.float8_e4m3fn else q_fp8
+    k8 = k_fp8.view(torch.uint8) if k_fp8.dtype == torch.float8_e4m3fn else k_fp8
+    _need(q8, torch.uint8, "q_fp8", 3)
+    _need(k8, torch.uint8, "k_fp8", 2)
+    _need(q, torch.bfloat16, "q", 3)
+    _need(kv, torch.bfloat16, "kv", 2)
+    _need(out, torch.bfloat16, "out", 3)
+    _need(lse, torch.float32, "lse", 2)
+    _need(idx_out, torch.int32, "idx_out", 2)
+    T_q, H_I, d_I = q8.shape
+    _, H, d_qk = q.shape
+    rc = load().dsa_forward_noalloc(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale),
+                                    _ptr(q), _ptr(kv), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+                                    int(B), int(max_len_q), int(max_len_k), int(T_q),
+                                    int(k8.shape[0]), int(H_I), int(d_I), int(H), int(d_qk),
+                                    int(out.shape[2]), int(k), float(sm_scale), _ptr(out),
+                                    _ptr(lse), _ptr(idx_out), _stream(stream))
+    _check(rc, "dsa_forward_noalloc")
 
 
 def dsa_get_device_error(stream=None) -> int:
