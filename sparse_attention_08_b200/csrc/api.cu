@@ -220,10 +220,6 @@ dsa_status_t dsa_sparse_mla_fwd(const void* q, const void* kv, const int32_t* id
   if (total_k == 0) return DSA_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;
   if ((st = device_info(&dev)) != DSA_OK) return st;
-  CUtensorMap tq;
-  if ((st = encode_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, total_q * H, 576, 2, 64, 64,
-                      CU_TENSOR_MAP_SWIZZLE_128B)) != DSA_OK)
-    return st;
   dsa::MlaArgs a;
   a.idx = idx;
   a.cu_q = cu_seqlens_q;
@@ -239,7 +235,7 @@ dsa_status_t dsa_sparse_mla_fwd(const void* q, const void* kv, const int32_t* id
   a.out = out;
   a.lse = lse;
   return from_cuda(
-      dsa::launch_sparse_mla(tq, kv, a, next_err(dev), static_cast<cudaStream_t>(stream)));
+      dsa::launch_sparse_mla(q, kv, a, next_err(dev), static_cast<cudaStream_t>(stream)));
 }
 
 size_t dsa_forward_workspace_size(int64_t total_q, int max_len_k, int k) {

@@ -35,8 +35,8 @@ constexpr int kBlockK = 128;      // keys per tile (MMA M)
 constexpr int kN = 256;           // MMA N = queries per tile * H_I
 constexpr int kKbPerItem = 16;    // key blocks per work item
 constexpr int kStages = 6;        // key-tile pipeline depth
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
+constexpr int kThreads = 320;      // producer, MMA, two epilogue warpgroups
+constexpr int kEpiThreads = 128;   // one epilogue warpgroup
 constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
 
 struct Params {
@@ -97,7 +97,7 @@ struct Layout {
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffK = kOffQ + 2 * kQBytes;
   static constexpr uint32_t kOffWq = kOffK + kStages * kKBytes;
-  static constexpr uint32_t kOffBar = kOffWq + kN * 4;
+  static constexpr uint32_t kOffBar = kOffWq + 2 * kN * 4;     // one wq copy per warpgroup
   // barriers: q_full[2], q_empty[2], k_full[S], k_empty[S], acc_full[2], acc_empty[2], drain
   static constexpr uint32_t kNumBars = 2 + 2 + kStages + kStages + 2 + 2 + 1;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
@@ -234,17 +234,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int et = threadIdx.x - 64;          // 0..127
+    // Two warpgroups take alternate tiles (accumulator buffer eg), so one
+    // group's TMEM loads overlap the other's arithmetic.  Warp w reads TMEM
+    // lanes 32*(w%4)..; a thread owns one key of the tile.
+    const int eg = (warp - 2) >> 2;            // warpgroup 0 or 1
+    const int et = threadIdx.x - 64 - eg * kEpiThreads;   // 0..127 within the group
+    const uint32_t bar_id = 1 + eg;
     const int sp = warp & 3;                  // TMEM sub-partition of this warp
     const int row = sp * 32 + lane;           // TMEM lane = key within the tile
     const uint32_t lane_addr = static_cast<uint32_t>(sp * 32) << 16;
+    float* wq = wq_s + eg * kN;
+    // chunks of 32 columns loaded per tcgen05.wait (register budget)
+    constexpr int kChunksPerWait = QPT >= 32 ? 1 : 2;
     int64_t ac = 0;
     bool ok = true;
     for (int64_t item = blockIdx.x; ok && item < P.n_items; item += gridDim.x) {
       Item it;
       if (!decode_item<QPT>(item, P, it)) continue;
       // head weights of this query group: wq[qi*H_I + j] = w * q_scale
-      named_bar_sync(1, kEpiThreads);
+      named_bar_sync(bar_id, kEpiThreads);
       for (int n = et; n < kN; n += kEpiThreads) {
         const int qi = n / H_I;
         float v = 0.f;
@@ -252,49 +260,57 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int64_t o = static_cast<int64_t>(it.q_row0 + qi) * H_I + (n % H_I);
           v = __ldg(P.w + o) * __ldg(P.q_scale + o);
         }
-        wq_s[n] = v;
+        wq[n] = v;
       }
-      named_bar_sync(1, kEpiThreads);
-      for (int j = 0; j < it.nkb; ++j) {
+      named_bar_sync(bar_id, kEpiThreads);
+      for (int j = 0; j < it.nkb; ++j, ++ac) {
         const int ab = static_cast<int>(ac & 1);
+        if (ab != eg) continue;
         if (et == 0) {
           if (!mbar_wait(acc_full(ab), static_cast<uint32_t>((ac >> 1) & 1), P.err)) *abort_flag = 1;
         }
-        named_bar_sync(1, kEpiThreads);
+        named_bar_sync(bar_id, kEpiThreads);
         if (*abort_flag) {
           ok = false;
           break;
         }
         tc_fence_after();
         const int s_local = (it.kb0 + j) * kBlockK + row;
-        float acc[QPT];
+        // two running sums per query (even / odd heads) for the packed FMA
+        float2 acc[QPT];
 #pragma unroll
-        for (int qi = 0; qi < QPT; ++qi) acc[qi] = 0.f;
+        for (int qi = 0; qi < QPT; ++qi) acc[qi] = make_float2(0.f, 0.f);
         const uint32_t dcol = tmem + lane_addr + static_cast<uint32_t>(ab) * kN;
 #pragma unroll
-        for (int ch = 0; ch < kN / 32; ++ch) {
-          if ((ch * 32) / H_I < it.nq) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(dcol + ch * 32, v);
-            tmem_wait_ld();
+        for (int cg = 0; cg < kN / 32; cg += kChunksPerWait) {
+          if ((cg * 32) / H_I >= it.nq) break;
+          uint32_t v[kChunksPerWait][32];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const int n = ch * 32 + c;
-              acc[n / H_I] = fmaf(wq_s[n], fmaxf(__uint_as_float(v[c]), 0.f), acc[n / H_I]);
+          for (int u = 0; u < kChunksPerWait; ++u) tmem_ld_32x32b_x32(dcol + (cg + u) * 32, v[u]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < kChunksPerWait; ++u) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              const int n = (cg + u) * 32 + c;
+              const float2 w2 = *reinterpret_cast<const float2*>(wq + n);
+              const float2 x2 = make_float2(fmaxf(__uint_as_float(v[u][c]), 0.f),
+                                            fmaxf(__uint_as_float(v[u][c + 1]), 0.f));
+              acc[n / H_I] = __ffma2_rn(w2, x2, acc[n / H_I]);
             }
           }
         }
         tc_fence_before();
-        named_bar_sync(1, kEpiThreads);
+        named_bar_sync(bar_id, kEpiThreads);
         if (et == 0) mbar_arrive(acc_empty(ab));
-        ++ac;
         if (s_local < it.len_k) {
           const float ks = __ldg(P.k_scale + it.k_row0 + s_local);
           const int p0 = it.len_k - it.len_q + it.q0;
 #pragma unroll
           for (int qi = 0; qi < QPT; ++qi) {
             if (qi < it.nq && s_local <= p0 + qi)
-              P.logits[static_cast<int64_t>(it.q_row0 + qi) * P.ld + s_local] = acc[qi] * ks;
+              P.logits[static_cast<int64_t>(it.q_row0 + qi) * P.ld + s_local] =
+                  (acc[qi].x + acc[qi].y) * ks;
           }
         }
       }

@@ -50,7 +50,7 @@ struct MlaArgs {
 cudaError_t launch_indexer(const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
                            const IndexerArgs& a, int num_sms, DevErr err, cudaStream_t s);
 cudaError_t launch_topk(const TopkArgs& a, DevErr err, cudaStream_t s);
-cudaError_t launch_sparse_mla(const CUtensorMap& tmap_q, const void* kv, const MlaArgs& a,
-                              DevErr err, cudaStream_t s);
+cudaError_t launch_sparse_mla(const void* q, const void* kv, const MlaArgs& a, DevErr err,
+                              cudaStream_t s);
 
 }  // namespace dsa
