@@ -108,7 +108,8 @@ DSA_API dsa_status_t dsa_indexer_logits(const void* q_fp8, const float* q_scale,
  * ascending position order, padded with -1.  Ties go to the lower position;
  * -0.0 and +0.0 are equal.  NaN scores are not supported.
  *
- *  logits   (device) f32, layout as produced by dsa_indexer_logits
+ *  logits   (device) f32, layout as produced by dsa_indexer_logits (16-byte
+ *           aligned, ld_logits a multiple of 4, else DSA_ERR_ALIGNMENT)
  *  idx_out  (device) int32 [total_q, k]
  *  val_out  (device, nullable) f32 [total_q, k]: the selected scores (NaN in
  *           padding slots)

@@ -176,7 +176,8 @@ dsa_status_t dsa_topk(const float* logits, int64_t ld_logits, const int32_t* cu_
   if (k < 1 || k > 4096) return DSA_ERR_UNSUPPORTED;
   if (max_len_k > (1 << 24)) return DSA_ERR_UNSUPPORTED;
   if (ld_logits < max_len_k || ld_logits < 1) return DSA_ERR_INVALID_ARG;
-  if (!aligned16(logits) || !aligned16(idx_out) || (val_out && !aligned16(val_out)))
+  if (!aligned16(logits) || !aligned16(idx_out) || (val_out && !aligned16(val_out)) ||
+      (ld_logits % 4) != 0)
     return DSA_ERR_ALIGNMENT;
   if (total_q >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
   if (total_q == 0 || B == 0) return DSA_OK;

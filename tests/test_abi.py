@@ -80,6 +80,7 @@ def test_topk_and_attention_argument_checks():
     assert lib.dsa_topk(p, 64, p, p, 1, 64, 64, 64, 5000, p, None, None) == UNSUPPORTED
     assert lib.dsa_topk(None, 64, p, p, 1, 64, 64, 64, 16, p, None, None) == INVALID
     assert lib.dsa_topk(p, 64, p, p, 1, 64, 64, 64, 16, _fake(0x10008), None, None) == ALIGN
+    assert lib.dsa_topk(p, 66, p, p, 1, 64, 64, 64, 16, p, None, None) == ALIGN
     f = ctypes.c_float(1.0 / 24)
     mla = lib.dsa_sparse_mla_fwd
     assert mla(p, p, p, p, p, 1, 64, 64, 64, 64, 128, 512, 512, 64, f, p, None, None) == UNSUPPORTED
