@@ -12,16 +12,24 @@
 //   D[s, (t,j)] = sum_d k8[s,d] * q8[t,j,d],     M = 128 keys, N = 256 = QPT*H_I,
 // issued as tcgen05.mma kind::f8f6f4 (e4m3 x e4m3 -> f32) from TMA-fed,
 // 128/64-byte-swizzled shared-memory tiles into a double-buffered TMEM
-// accumulator.  Four epilogue warps own one key (TMEM lane) each and fold
+// accumulator.  Epilogue threads own one key (TMEM lane) each and fold
 // ReLU, the (w * q_scale) head weights, the k_scale multiply and the causal
 // mask into the read-out, so no per-head score ever leaves the SM.
 //
 // Work items: (sequence, group of QPT queries, chunk of KB_PER_ITEM key
 // blocks) on a persistent grid of one CTA per SM, strided over a virtual item
 // space; items outside the causal triangle are skipped by every role alike.
+// The number of virtual key chunks is padded to be coprime with the grid, so
+// that every CTA's stride visits every chunk index alike: chunks far from
+// the diagonal are skipped more often, and a CTA that only ever saw them
+// would finish early.
 //
-// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM owner and
-// MMA issuer, warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4)..).
+// Warp roles (576 threads): warp 0 = TMA producer, warp 1 = TMEM owner and
+// MMA issuer, warps 2..17 = four epilogue warpgroups.  Warpgroup g reads
+// accumulator buffer g/2 and the column half g%2 (half of the tile's
+// queries); warp w reads TMEM lanes 32*(w%4)...  The ReLU / weighted-sum
+// read-out costs about as many issue slots as the MMA takes cycles, so it
+// is spread over four warps per sub-partition to hide TMEM and FMA latency.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -35,8 +43,9 @@ constexpr int kBlockK = 128;      // keys per tile (MMA M)
 constexpr int kN = 256;           // MMA N = queries per tile * H_I
 constexpr int kKbPerItem = 16;    // key blocks per work item
 constexpr int kStages = 6;        // key-tile pipeline depth
-constexpr int kThreads = 320;      // producer, MMA, two epilogue warpgroups
+constexpr int kEpiGroups = 4;
 constexpr int kEpiThreads = 128;   // one epilogue warpgroup
+constexpr int kThreads = 64 + kEpiGroups * kEpiThreads;   // producer, MMA, epilogue
 constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
 
 struct Params {
@@ -97,7 +106,7 @@ struct Layout {
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffK = kOffQ + 2 * kQBytes;
   static constexpr uint32_t kOffWq = kOffK + kStages * kKBytes;
-  static constexpr uint32_t kOffBar = kOffWq + 2 * kN * 4;     // one wq copy per warpgroup
+  static constexpr uint32_t kOffBar = kOffWq + kEpiGroups * (kN / 2) * 4;  // wq half per warpgroup
   // barriers: q_full[2], q_empty[2], k_full[S], k_empty[S], acc_full[2], acc_empty[2], drain
   static constexpr uint32_t kNumBars = 2 + 2 + kStages + kStages + 2 + 2 + 1;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
@@ -138,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(q_full(i), 1);
       mbar_init(q_empty(i), 1);
       mbar_init(acc_full(i), 1);
-      mbar_init(acc_empty(i), 1);
+      mbar_init(acc_empty(i), 2);     // both column halves read the buffer
     }
     for (int i = 0; i < kStages; ++i) {
       mbar_init(k_full(i), 1);
@@ -234,30 +243,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // Two warpgroups take alternate tiles (accumulator buffer eg), so one
-    // group's TMEM loads overlap the other's arithmetic.  Warp w reads TMEM
-    // lanes 32*(w%4)..; a thread owns one key of the tile.
-    const int eg = (warp - 2) >> 2;            // warpgroup 0 or 1
+    // Warpgroup eg reads accumulator buffer eg/2 (every other tile) and the
+    // column half eg%2.  Warp w reads TMEM lanes 32*(w%4)..; a thread owns
+    // one key of the tile.
+    const int eg = (warp - 2) >> 2;            // warpgroup 0..3
+    const int ab_mine = eg >> 1;
+    const int hf = eg & 1;
     const int et = threadIdx.x - 64 - eg * kEpiThreads;   // 0..127 within the group
     const uint32_t bar_id = 1 + eg;
     const int sp = warp & 3;                  // TMEM sub-partition of this warp
     const int row = sp * 32 + lane;           // TMEM lane = key within the tile
     const uint32_t lane_addr = static_cast<uint32_t>(sp * 32) << 16;
-    float* wq = wq_s + eg * kN;
+    constexpr int kHalf = kN / 2;             // columns per warpgroup
+    constexpr int QH = QPT / 2;               // queries per warpgroup
+    // independent FMA chains per query (latency hiding)
+    constexpr int NCH = H_I >= 16 ? 4 : (H_I >= 8 ? 2 : 1);
     // chunks of 32 columns loaded per tcgen05.wait (register budget)
-    constexpr int kChunksPerWait = QPT >= 32 ? 1 : 2;
+    constexpr int kChunksPerWait = 1;
+    float* wq = wq_s + eg * kHalf;
     int64_t ac = 0;
     bool ok = true;
     for (int64_t item = blockIdx.x; ok && item < P.n_items; item += gridDim.x) {
       Item it;
       if (!decode_item<QPT>(item, P, it)) continue;
-      // head weights of this query group: wq[qi*H_I + j] = w * q_scale
+      // head weights of this half of the query group: w * q_scale
       named_bar_sync(bar_id, kEpiThreads);
-      for (int n = et; n < kN; n += kEpiThreads) {
-        const int qi = n / H_I;
+      for (int n = et; n < kHalf; n += kEpiThreads) {
+        const int col = hf * kHalf + n;
+        const int qi = col / H_I;
         float v = 0.f;
         if (qi < it.nq) {
-          const int64_t o = static_cast<int64_t>(it.q_row0 + qi) * H_I + (n % H_I);
+          const int64_t o = static_cast<int64_t>(it.q_row0 + qi) * H_I + (col % H_I);
           v = __ldg(P.w + o) * __ldg(P.q_scale + o);
         }
         wq[n] = v;
@@ -265,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar_sync(bar_id, kEpiThreads);
       for (int j = 0; j < it.nkb; ++j, ++ac) {
         const int ab = static_cast<int>(ac & 1);
-        if (ab != eg) continue;
+        if (ab != ab_mine) continue;
         if (et == 0) {
           if (!mbar_wait(acc_full(ab), static_cast<uint32_t>((ac >> 1) & 1), P.err)) *abort_flag = 1;
         }
@@ -276,14 +292,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const int s_local = (it.kb0 + j) * kBlockK + row;
-        // two running sums per query (even / odd heads) for the packed FMA
-        float2 acc[QPT];
+        float2 acc[QH][NCH];
 #pragma unroll
-        for (int qi = 0; qi < QPT; ++qi) acc[qi] = make_float2(0.f, 0.f);
-        const uint32_t dcol = tmem + lane_addr + static_cast<uint32_t>(ab) * kN;
+        for (int qi = 0; qi < QH; ++qi) {
 #pragma unroll
-        for (int cg = 0; cg < kN / 32; cg += kChunksPerWait) {
-          if ((cg * 32) / H_I >= it.nq) break;
+          for (int ch = 0; ch < NCH; ++ch) acc[qi][ch] = make_float2(0.f, 0.f);
+        }
+        const uint32_t dcol = tmem + lane_addr + static_cast<uint32_t>(ab) * kN + hf * kHalf;
+#pragma unroll
+        for (int cg = 0; cg < kHalf / 32; cg += kChunksPerWait) {
+          if ((hf * kHalf + cg * 32) / H_I >= it.nq) break;
           uint32_t v[kChunksPerWait][32];
 #pragma unroll
           for (int u = 0; u < kChunksPerWait; ++u) tmem_ld_32x32b_x32(dcol + (cg + u) * 32, v[u]);
@@ -291,12 +309,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int u = 0; u < kChunksPerWait; ++u) {
 #pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-              const int n = (cg + u) * 32 + c;
-              const float2 w2 = *reinterpret_cast<const float2*>(wq + n);
-              const float2 x2 = make_float2(fmaxf(__uint_as_float(v[u][c]), 0.f),
-                                            fmaxf(__uint_as_float(v[u][c + 1]), 0.f));
-              acc[n / H_I] = __ffma2_rn(w2, x2, acc[n / H_I]);
+            for (int c = 0; c < 32; c += 4) {
+              const int n = (cg + u) * 32 + c;          // column within the half
+              const int ql = n / H_I;                   // query within the half
+              const int ch = ((n % H_I) / 4) % NCH;
+              const float4 w4 = *reinterpret_cast<const float4*>(wq + n);
+              const float2 x01 = make_float2(fmaxf(__uint_as_float(v[u][c]), 0.f),
+                                             fmaxf(__uint_as_float(v[u][c + 1]), 0.f));
+              const float2 x23 = make_float2(fmaxf(__uint_as_float(v[u][c + 2]), 0.f),
+                                             fmaxf(__uint_as_float(v[u][c + 3]), 0.f));
+              acc[ql][ch] = __ffma2_rn(make_float2(w4.x, w4.y), x01, acc[ql][ch]);
+              acc[ql][ch] = __ffma2_rn(make_float2(w4.z, w4.w), x23, acc[ql][ch]);
             }
           }
         }
@@ -307,10 +330,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float ks = __ldg(P.k_scale + it.k_row0 + s_local);
           const int p0 = it.len_k - it.len_q + it.q0;
 #pragma unroll
-          for (int qi = 0; qi < QPT; ++qi) {
+          for (int ql = 0; ql < QH; ++ql) {
+            const int qi = hf * QH + ql;
+            float sum = 0.f;
+#pragma unroll
+            for (int ch = 0; ch < NCH; ++ch) sum += acc[ql][ch].x + acc[ql][ch].y;
             if (qi < it.nq && s_local <= p0 + qi)
-              P.logits[static_cast<int64_t>(it.q_row0 + qi) * P.ld + s_local] =
-                  (acc[qi].x + acc[qi].y) * ks;
+              P.logits[static_cast<int64_t>(it.q_row0 + qi) * P.ld + s_local] = sum * ks;
           }
         }
       }
@@ -343,11 +369,24 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const Indexer
   P.n_items = static_cast<int64_t>(a.B) * P.n_qg * P.n_kc;
   P.err = err;
   if (P.n_items == 0) return cudaSuccess;
+  const int64_t grid = P.n_items < num_sms ? P.n_items : num_sms;
+  // Virtual key chunks past the last one are skipped like any chunk outside
+  // the causal triangle; padding their count to be coprime with the grid
+  // makes each CTA's stride cycle through every chunk index.
+  auto gcd = [](int64_t x, int64_t y) {
+    while (y) {
+      const int64_t t = x % y;
+      x = y;
+      y = t;
+    }
+    return x;
+  };
+  while (gcd(P.n_kc, grid) != 1) ++P.n_kc;
+  P.n_items = static_cast<int64_t>(a.B) * P.n_qg * P.n_kc;
   auto kern = indexer_kernel<H_I, D_I>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(L::kSmem));
   if (e != cudaSuccess) return e;
-  const int64_t grid = P.n_items < num_sms ? P.n_items : num_sms;
   kern<<<static_cast<unsigned>(grid), kThreads, L::kSmem, s>>>(tq, tk, P);
   return cudaGetLastError();
 }
