@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(q_full(i), 1);
       mbar_init(q_empty(i), 1);
       mbar_init(acc_full(i), 1);
-      mbar_init(acc_empty(i), 2);     // both column halves read the buffer
+      mbar_init(acc_empty(i), 8);     // every warp of both column halves reads the buffer
     }
     for (int i = 0; i < kStages; ++i) {
       mbar_init(k_full(i), 1);
@@ -282,11 +282,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < it.nkb; ++j, ++ac) {
         const int ab = static_cast<int>(ac & 1);
         if (ab != ab_mine) continue;
-        if (et == 0) {
-          if (!mbar_wait(acc_full(ab), static_cast<uint32_t>((ac >> 1) & 1), P.err)) *abort_flag = 1;
-        }
-        named_bar_sync(bar_id, kEpiThreads);
-        if (*abort_flag) {
+        // each warp waits and releases on its own: no warpgroup barrier per tile
+        if (!warp_wait(acc_full(ab), static_cast<uint32_t>((ac >> 1) & 1), P.err)) {
+          *abort_flag = 1;
           ok = false;
           break;
         }
@@ -324,8 +322,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tc_fence_before();
-        named_bar_sync(bar_id, kEpiThreads);
-        if (et == 0) mbar_arrive(acc_empty(ab));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty(ab));
         if (s_local < it.len_k) {
           const float ks = __ldg(P.k_scale + it.k_row0 + s_local);
           const int p0 = it.len_k - it.len_q + it.q0;
