@@ -235,6 +235,7 @@ dsa_status_t dsa_sparse_mla_fwd(const void* q, const void* kv, const int32_t* id
   a.sm_scale = sm_scale;
   a.out = out;
   a.lse = lse;
+  a.num_sms = dev->num_sms;
   return from_cuda(
       dsa::launch_sparse_mla(q, kv, a, next_err(dev), static_cast<cudaStream_t>(stream)));
 }

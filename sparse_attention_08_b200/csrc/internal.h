@@ -44,6 +44,7 @@ struct MlaArgs {
   float sm_scale;
   void* out;
   float* lse;
+  int num_sms;   // persistent grid size
 };
 
 // Each returns cudaSuccess or the launch error.

@@ -235,6 +235,20 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
       : "memory");
 }
 
+// True in exactly one lane of a converged warp (the lowest active lane).
+// Issuing a run of tcgen05 instructions inside one elected block keeps the
+// code compact: an elect per instruction makes the compiler materialise each
+// operand separately, which multiplies the size of long unrolled MMA runs.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, e;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // Warp-wide forms: the whole warp executes them with converged control flow
 // and one elected lane issues.  Issued this way (every operand warp-uniform)
 // back-to-back MMAs reach the tensor pipe without per-instruction gaps.
