@@ -490,25 +490,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free(sb));
 
-        // key of register 4i+e (row a) and 4i+2+e (row b): 8i + 2qd + e
+        // key of register 4i+e (row a) and 4i+2+e (row b): 8i + 2qd + e.
+        // Entries outside the selection get the raw score -inf; full blocks
+        // (all but the last block of short rows) skip the masking.
+        if ((vmask_lo & vmask_hi) != 0xffffffffu) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              if (!((((e ? vmask_hi : vmask_lo) >> (4 * i + qd)) & 1u) != 0)) {
+                v[4 * i + e] = 0xff800000u;
+                v[4 * i + 2 + e] = 0xff800000u;
+              }
+            }
+          }
+        }
+        // row maxima on the raw scores (the scale is positive), in log2 units
         float mxa = -INFINITY, mxb = -INFINITY;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const bool valid = (((e ? vmask_hi : vmask_lo) >> (4 * i + qd)) & 1u) != 0;
-            const float xa = valid ? __uint_as_float(v[4 * i + e]) * P.scale_log2 : -INFINITY;
-            const float xb = valid ? __uint_as_float(v[4 * i + 2 + e]) * P.scale_log2 : -INFINITY;
-            v[4 * i + e] = __float_as_uint(xa);
-            v[4 * i + 2 + e] = __float_as_uint(xb);
-            mxa = fmaxf(mxa, xa);
-            mxb = fmaxf(mxb, xb);
-          }
+          mxa = fmaxf(mxa, fmaxf(__uint_as_float(v[4 * i + 0]), __uint_as_float(v[4 * i + 1])));
+          mxb = fmaxf(mxb, fmaxf(__uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3])));
         }
         mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
         mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
         mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
         mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
+        mxa *= P.scale_log2;
+        mxb *= P.scale_log2;
         float al_a = 1.f, al_b = 1.f;
         bool moved = false;
         if (mxa > m_a + kRescaleThreshold) {
@@ -523,31 +532,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const bool rescale = j > 0 && __any_sync(0xffffffffu, moved);
 
-        // P (bf16) over the slot's RoPE chunk: row r, keys 8i..8i+7 are the
-        // 16-byte piece i, stored at piece i ^ (r & 7).
+        // P = exp2(scale * s - m) (bf16) over the slot's RoPE chunk: row r,
+        // keys 8i..8i+7 are the 16-byte piece i, stored at piece i ^ (r & 7).
+        // A row with no entry yet (m = -inf) has only -inf scores: p = 0.
+        const float nma = m_a == -INFINITY ? 0.f : -m_a;
+        const float nmb = m_b == -INFINITY ? 0.f : -m_b;
         uint8_t* pst = smem + kOffKv + st * kKvBytes + kOffPInStage;
-        float sa = 0.f, sb_ = 0.f, sra = 0.f, srb = 0.f;
+        // two sums per row, as packed pairs: of the fp32 probabilities (for
+        // the lse) and of the bf16-rounded ones the MMA consumes (O is
+        // normalised by these, so its weights sum to one exactly)
+        float2 s2a = make_float2(0.f, 0.f), s2b = s2a, r2a = s2a, r2b = s2a;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float xa0 = __uint_as_float(v[4 * i + 0]), xa1 = __uint_as_float(v[4 * i + 1]);
-          const float xb0 = __uint_as_float(v[4 * i + 2]), xb1 = __uint_as_float(v[4 * i + 3]);
-          const float pa0 = xa0 == -INFINITY ? 0.f : fast_exp2(xa0 - m_a);
-          const float pa1 = xa1 == -INFINITY ? 0.f : fast_exp2(xa1 - m_a);
-          const float pb0 = xb0 == -INFINITY ? 0.f : fast_exp2(xb0 - m_b);
-          const float pb1 = xb1 == -INFINITY ? 0.f : fast_exp2(xb1 - m_b);
-          sa += pa0 + pa1;
-          sb_ += pb0 + pb1;
+          const float pa0 = fast_exp2(fmaf(__uint_as_float(v[4 * i + 0]), P.scale_log2, nma));
+          const float pa1 = fast_exp2(fmaf(__uint_as_float(v[4 * i + 1]), P.scale_log2, nma));
+          const float pb0 = fast_exp2(fmaf(__uint_as_float(v[4 * i + 2]), P.scale_log2, nmb));
+          const float pb1 = fast_exp2(fmaf(__uint_as_float(v[4 * i + 3]), P.scale_log2, nmb));
+          s2a = __fadd2_rn(s2a, make_float2(pa0, pa1));
+          s2b = __fadd2_rn(s2b, make_float2(pb0, pb1));
           const uint32_t ka = pack_bf16x2(pa0, pa1), kb = pack_bf16x2(pb0, pb1);
-          // the weights O receives are the rounded ones: normalise by their sum
-          sra += __uint_as_float(ka << 16) + __uint_as_float(ka & 0xFFFF0000u);
-          srb += __uint_as_float(kb << 16) + __uint_as_float(kb & 0xFFFF0000u);
+          r2a = __fadd2_rn(r2a, make_float2(__uint_as_float(ka << 16), __uint_as_float(ka & 0xFFFF0000u)));
+          r2b = __fadd2_rn(r2b, make_float2(__uint_as_float(kb << 16), __uint_as_float(kb & 0xFFFF0000u)));
           *reinterpret_cast<uint32_t*>(pst + ra * 128 + ((i ^ (ra & 7)) << 4) + 4 * qd) = ka;
           *reinterpret_cast<uint32_t*>(pst + rb * 128 + ((i ^ (rb & 7)) << 4) + 4 * qd) = kb;
         }
-        l_a = l_a * al_a + sa;
-        l_b = l_b * al_b + sb_;
-        lr_a = lr_a * al_a + sra;
-        lr_b = lr_b * al_b + srb;
+        l_a = l_a * al_a + (s2a.x + s2a.y);
+        l_b = l_b * al_b + (s2b.x + s2b.y);
+        lr_a = lr_a * al_a + (r2a.x + r2a.y);
+        lr_b = lr_b * al_b + (r2b.x + r2b.y);
 
         // When a maximum moved, this warp's O rows are rescaled before P V of
         // this block may run: after P V of the previous block has completed
