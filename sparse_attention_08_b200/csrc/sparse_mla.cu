@@ -31,14 +31,16 @@
 //    needs, so P lives and dies with its slot.
 //  * warps 0..3 (softmax): each owns 16 heads and all 32 lanes work: the
 //    16x256b TMEM access shape gives lane t the rows t/4 and 8+t/4 of the
-//    warp's 16, two adjacent columns of every group of 8.  Per item they
-//    move the query tile into TMEM; per block they read S, run the online
-//    softmax in fp32 (exp2, lazily rescaled maximum), write P (bf16) to
-//    shared memory and rescale their own O rows in TMEM when their maximum
-//    moves; at the end of an item they hand the row statistics on.
-//  * warps 9..12 (output): once an item's last product has landed, normalise
-//    O and store bf16 out (16-byte stores after a 4 x 4 shuffle transpose)
-//    and the lse, then hand the accumulator back for the next item.
+//    warp's 16, two adjacent columns of every group of 8.  Per block they
+//    read S, run the online softmax in fp32 (exp2, lazily rescaled maximum),
+//    write P (bf16) to shared memory and rescale their own O rows in TMEM
+//    when their maximum moves; at the end of an item they hand the row
+//    statistics on.
+//  * warps 9..12 (output, same lane mapping): move each item's query tile
+//    from its ring slot into TMEM (as soon as the previous item's last S
+//    is done), and once an item's last product has landed, normalise O and
+//    store bf16 out (16-byte stores after a 4 x 4 shuffle transpose) and the
+//    lse, handing the accumulator back after its last chunk is loaded.
 //
 // TMEM (512 columns x 128 lanes): an M=64 accumulator fills lanes 0-15 of
 // each 32-lane sub-partition; a second one at lane offset 16 fills lanes
@@ -71,8 +73,8 @@ constexpr uint32_t kOffPInStage = 8 * kChunkBytes;    // P (64 x 64 bf16) over t
 constexpr int kStatRing = 4;                      // row statistics of items in flight
 constexpr uint32_t kOffBar = kOffKv + kStages * kKvBytes;
 // barriers: kv_full[S], kv_empty[S], p_full[S], s_full[2], s_free[2],
-// q_ready, o_full, o_free, stats_full[kStatRing], drain[2]
-constexpr uint32_t kNumBars = 3 * kStages + 4 + 3 + kStatRing + 2;
+// q_ready, o_full, o_free, stats_full[kStatRing], drain[2], s_last
+constexpr uint32_t kNumBars = 3 * kStages + 4 + 3 + kStatRing + 2 + 1;
 constexpr uint32_t kOffStats = (kOffBar + kNumBars * 8 + 15) & ~15u;   // [kStatRing][64][4] floats
 constexpr uint32_t kOffMisc = kOffStats + kStatRing * kHeads * 4 * 4;
 constexpr uint32_t kSmem = kOffMisc + 32 + 1024;
@@ -211,6 +213,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t o_free = bar0 + 8u * (3 * kStages + 6);    // O read out
   auto stats_full = [&](uint32_t i) { return bar0 + 8u * (3 * kStages + 7 + i); };
   auto drain_bar = [&](uint32_t i) { return bar0 + 8u * (3 * kStages + 7 + kStatRing + i); };
+  // last S of an item done: one phase per item, so a waiter that is an item
+  // ahead of the score products can never see a stale phase
+  const uint32_t s_last = bar0 + 8u * (3 * kStages + 9 + kStatRing);
   float* stats = reinterpret_cast<float*>(smem + kOffStats);      // [ring][row][m, l, lr, -]
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
@@ -235,6 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kStatRing; ++i) mbar_init(stats_full(i), kSmWarps);
     mbar_init(drain_bar(0), 1);
     mbar_init(drain_bar(1), 1);
+    mbar_init(s_last, 1);
     *abort_flag = 0;
     *q_reads = 0u;
     fence_barrier_init();
@@ -359,6 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           mma_commit(s_full(sb));
+          if (c.j + 1 == c.it.nb) mma_commit(s_last);
         }
         __syncwarp();
         cursor_next(c, P);
@@ -411,72 +418,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(w * 32) << 16;
     bool ok = true;
     uint32_t u = 0, gb = 0, ii = 0;
+    // Validity of block entries: lane l checks entries 2l and 2l+1.
+    auto entry_ok = [&](const Item& x, int e) -> bool {
+      if (e >= x.n_sel) return false;
+      const int s = __ldg(P.idx + x.q_row * P.k + e);
+      return s >= 0 && s <= x.p;
+    };
+    // The next item's bookkeeping (its global loads) is done one item ahead,
+    // off the path from the last block of an item to the first of the next.
+    Item it = item_at(P, blockIdx.x);
+    bool nx0 = entry_ok(it, 2 * lane), nx1 = entry_ok(it, 2 * lane + 1);
     for (int64_t wi = blockIdx.x; ok && wi < P.n_items; wi += gridDim.x, ++ii) {
-      const Item it = item_at(P, wi);
-      const int32_t* idx_row = P.idx + it.q_row * P.k;
-      // ---- query tile: ring slot -> TMEM columns kQCol.., lanes 16..31.
-      // Column 32c+8i+2qd+e holds elements 64c+16i+4qd+2e, +1 of a row.  All
-      // S products of the previous item are complete (their scores were read).
-      {
-        const uint32_t st = u % kStages;
-        if (!warp_wait(kv_full(st), (u / kStages) & 1, P.err)) {
-          ok = false;
-          break;
-        }
-        const uint8_t* qs = smem + kOffKv + st * kKvBytes;
-#pragma unroll 3
-        for (int c = 0; c < kChunks; ++c) {
-          uint32_t r[16];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int pc = 2 * i + (qd >> 1);
-            const uint2 va = *reinterpret_cast<const uint2*>(
-                qs + c * kChunkBytes + ra * 128 + ((pc ^ (ra & 7)) << 4) + 8 * (qd & 1));
-            const uint2 vb = *reinterpret_cast<const uint2*>(
-                qs + c * kChunkBytes + rb * 128 + ((pc ^ (rb & 7)) << 4) + 8 * (qd & 1));
-            r[4 * i + 0] = va.x;
-            r[4 * i + 1] = va.y;
-            r[4 * i + 2] = vb.x;
-            r[4 * i + 3] = vb.y;
-          }
-          tmem_st_16x256b_x4(tmem_q + lane_base + 32u * c, r);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          // The fourth warp to finish reading hands the slot back.  This
-          // comes before q_ready: once q_ready completes, every warp has
-          // counted itself, so the counter is back at zero for the next item.
-          if (atomicAdd(q_reads, 1u) == kSmWarps - 1) {
-            *q_reads = 0u;
-            mbar_arrive(kv_empty(st));
-          }
-          // every slot completes one phase of each of its barriers, so the
-          // phase parities stay a function of the slot number alone
-          mbar_arrive(p_full(st));
-          mbar_arrive(q_ready);
-        }
-        ++u;
-      }
+      ++u;                                      // the item's query slot (output warps)
       float m_a = -INFINITY, m_b = -INFINITY;   // running maxima, log2 units
       float l_a = 0.f, l_b = 0.f;               // partial denominators (fp32 probabilities), lse
       float lr_a = 0.f, lr_b = 0.f;             // partial denominators of the bf16 P, for O
-      // Validity of block entries: lane l checks entries 2l and 2l+1.
-      auto entry_ok = [&](int e) -> bool {
-        if (e >= it.n_sel) return false;
-        const int s = __ldg(idx_row + e);
-        return s >= 0 && s <= it.p;
-      };
-      bool nx0 = entry_ok(2 * lane), nx1 = entry_ok(2 * lane + 1);
+      const int64_t wn = wi + gridDim.x;
+      Item nit = it;
+      if (wn < P.n_items) nit = item_at(P, wn);
       for (int j = 0; j < it.nb; ++j, ++u, ++gb) {
         const uint32_t sb = gb & 1;            // S buffer
         const uint32_t st = u % kStages;       // slot (P goes over its RoPE chunk)
         const uint32_t vmask_lo = __ballot_sync(0xffffffffu, nx0);
         const uint32_t vmask_hi = __ballot_sync(0xffffffffu, nx1);
         if (j + 1 < it.nb) {
-          nx0 = entry_ok((j + 1) * kBlockN + 2 * lane);
-          nx1 = entry_ok((j + 1) * kBlockN + 2 * lane + 1);
+          nx0 = entry_ok(it, (j + 1) * kBlockN + 2 * lane);
+          nx1 = entry_ok(it, (j + 1) * kBlockN + 2 * lane + 1);
+        } else if (wn < P.n_items) {
+          nx0 = entry_ok(nit, 2 * lane);
+          nx1 = entry_ok(nit, 2 * lane + 1);
         }
         if (!warp_wait(s_full(sb), (gb >> 1) & 1, P.err)) {
           ok = false;
@@ -610,25 +580,84 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(stats_full(ii % kStatRing));
+      it = nit;
     }
     if (!ok && lane == 0) *abort_flag = 1;
   } else {
     // ------------------------------------------------------------ output
+    // Per item: first move the next item's query tile into TMEM (as soon as
+    // the item's last S product is complete), then read out O.
     const int sp = warp & 3;                  // sub-partition (warps 9..12 -> 1,2,3,0)
     const int qd = lane & 3;
-    const int ra = 16 * sp + (lane >> 2);
+    const int ra = 16 * sp + (lane >> 2);     // this lane's two heads (rows) in the group
     const int rb = ra + 8;
     const uint32_t lane_base = static_cast<uint32_t>(sp * 32) << 16;
     bool ok = true;
-    uint32_t ii = 0;
+    // Query tile: ring slot uq -> TMEM columns kQCol.., lanes 16..31.
+    // Column 32c+8i+2qd+e holds elements 64c+16i+4qd+2e, +1 of a row.
+    auto copy_query = [&](uint32_t uq) -> bool {
+      const uint32_t st = uq % kStages;
+      if (!warp_wait(kv_full(st), (uq / kStages) & 1, P.err)) return false;
+      const uint8_t* qs = smem + kOffKv + st * kKvBytes;
+#pragma unroll 3
+      for (int c = 0; c < kChunks; ++c) {
+        uint32_t r[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int pc = 2 * i + (qd >> 1);
+          const uint2 va = *reinterpret_cast<const uint2*>(
+              qs + c * kChunkBytes + ra * 128 + ((pc ^ (ra & 7)) << 4) + 8 * (qd & 1));
+          const uint2 vb = *reinterpret_cast<const uint2*>(
+              qs + c * kChunkBytes + rb * 128 + ((pc ^ (rb & 7)) << 4) + 8 * (qd & 1));
+          r[4 * i + 0] = va.x;
+          r[4 * i + 1] = va.y;
+          r[4 * i + 2] = vb.x;
+          r[4 * i + 3] = vb.y;
+        }
+        tmem_st_16x256b_x4(tmem_q + lane_base + 32u * c, r);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        // The fourth warp to finish reading hands the slot back.  This comes
+        // before q_ready: once q_ready completes, every warp has counted
+        // itself, so the counter is back at zero for the next item.
+        if (atomicAdd(q_reads, 1u) == 3u) {
+          *q_reads = 0u;
+          mbar_arrive(kv_empty(st));
+        }
+        // every slot completes one phase of each of its barriers, so the
+        // phase parities stay a function of the slot number alone
+        mbar_arrive(p_full(st));
+        mbar_arrive(q_ready);
+      }
+      return true;
+    };
+    uint32_t u = 0, ii = 0;
+    Item it = item_at(P, blockIdx.x);
+    ok = copy_query(0);
     for (int64_t wi = blockIdx.x; ok && wi < P.n_items; wi += gridDim.x, ++ii) {
-      const Item it = item_at(P, wi);
+      u += 1 + it.nb;                          // the next item's query slot
+      const int64_t wn = wi + gridDim.x;
+      Item nit = it;
+      if (wn < P.n_items) {
+        nit = item_at(P, wn);
+        // the query region of TMEM is free once this item's last S is done
+        ok = warp_wait(s_last, ii & 1, P.err) && copy_query(u);
+        if (!ok) break;
+      }
       if (!warp_wait(stats_full(ii % kStatRing), (ii / kStatRing) & 1, P.err) ||
           !warp_wait(o_full, ii & 1, P.err)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      // O is read two chunks at a time: the load of the next chunk is in
+      // flight while the current one is converted and stored, and O is
+      // handed back as soon as the last chunk has landed in registers.
+      uint32_t oa_[32], ob_[32];
+      tmem_ld_16x256b_x8(tmem_o + lane_base, oa_);
       const float* sr = stats + (ii % kStatRing) * kHeads * 4;
       const float4 sa = *reinterpret_cast<const float4*>(sr + 4 * ra);
       const float4 sb = *reinterpret_cast<const float4*>(sr + 4 * rb);
@@ -636,23 +665,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_b = sb.z > 0.f ? 1.f / sb.z : 0.f;
       const int64_t head0 = it.q_row * P.H + it.hg * kHeads;
       const bool have_a = ra < it.heads_here, have_b = rb < it.heads_here;
-      if (P.lse && qd == 0) {
-        if (have_a) P.lse[head0 + ra] = sa.y > 0.f ? (sa.x + log2f(sa.y)) * 0.69314718055994531f : -INFINITY;
-        if (have_b) P.lse[head0 + rb] = sb.y > 0.f ? (sb.x + log2f(sb.y)) * 0.69314718055994531f : -INFINITY;
-      }
       __nv_bfloat16* oa = P.out + (head0 + ra) * kDv;
       __nv_bfloat16* ob = P.out + (head0 + rb) * kDv;
-#pragma unroll 1
-      for (int k8 = 0; k8 < kDv / 64; ++k8) {
-        uint32_t o[32];
-        tmem_ld_16x256b_x8(tmem_o + lane_base + 64u * k8, o);
-        tmem_wait_ld();
-        if (k8 == kDv / 64 - 1) {
-          // O has been read: the next item's first P V may overwrite it
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(o_free);
-        }
+      auto store_chunk = [&](const uint32_t (&o)[32], int k8) {
 #pragma unroll
         for (int uu = 0; uu < 2; ++uu) {
           // groups 4uu..4uu+3 (dims 64k8 + 32uu .. +31); after the transpose
@@ -672,7 +687,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (have_a) *reinterpret_cast<uint4*>(oa + dim) = make_uint4(pa[0], pa[1], pa[2], pa[3]);
           if (have_b) *reinterpret_cast<uint4*>(ob + dim) = make_uint4(pb[0], pb[1], pb[2], pb[3]);
         }
+      };
+#pragma unroll 1
+      for (int k2 = 0; k2 < kDv / 128; ++k2) {
+        tmem_wait_ld();
+        tmem_ld_16x256b_x8(tmem_o + lane_base + 64u * (2 * k2 + 1), ob_);
+        store_chunk(oa_, 2 * k2);
+        tmem_wait_ld();
+        if (k2 + 1 < kDv / 128) {
+          tmem_ld_16x256b_x8(tmem_o + lane_base + 64u * (2 * k2 + 2), oa_);
+        } else {
+          // O has been read: the next item's first P V may overwrite it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(o_free);
+        }
+        store_chunk(ob_, 2 * k2 + 1);
       }
+      if (P.lse && qd == 0) {
+        if (have_a) P.lse[head0 + ra] = sa.y > 0.f ? (sa.x + log2f(sa.y)) * 0.69314718055994531f : -INFINITY;
+        if (have_b) P.lse[head0 + rb] = sb.y > 0.f ? (sb.x + log2f(sb.y)) * 0.69314718055994531f : -INFINITY;
+      }
+      it = nit;
     }
     if (!ok && lane == 0) *abort_flag = 1;
   }
