@@ -154,6 +154,12 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* m, 
 // ---------------------------------------------------------------------------
 // cp.async (LDGSTS): 16-byte global -> shared copies, cached in L2 only.
 // ---------------------------------------------------------------------------
+// Starts pulling `bytes` (a multiple of 16, 16-byte aligned) of global
+// memory into L2 without waiting for it.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
 }

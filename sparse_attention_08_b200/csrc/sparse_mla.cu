@@ -287,6 +287,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const uint32_t stage = sbase + kOffKv + st * kKvBytes;
+        if (j < 0 && tg == 0 && w + gridDim.x < P.n_items) {
+          // the next item's query rows come from HBM: start them towards L2 now,
+          // an item ahead of their slot
+          const Item nx = item_at(P, w + gridDim.x);
+          prefetch_l2_bulk(P.q + (nx.q_row * P.H + nx.hg * kHeads) * kDqk,
+                           static_cast<uint32_t>(nx.heads_here) * kDqk * 2u);
+        }
         if (j < 0) {
           // the query rows of the head group; rows past the last head are zero
           const __nv_bfloat16* q_grp = P.q + (it.q_row * P.H + it.hg * kHeads) * kDqk;
