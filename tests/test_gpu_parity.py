@@ -58,6 +58,23 @@ def test_indexer_real_varlen_and_chunk(H_I, d_I):
             assert np.all(np.isnan(g[q0 + r, p + 1:cpu.max_len_k]))
 
 
+@pytest.mark.parametrize("H_I,d_I,integer", [(64, 128, True), (128, 64, True), (32, 128, False),
+                                              (64, 64, False)])
+def test_indexer_decode_batch(H_I, d_I, integer):
+    # one query per sequence (the decode shape: one-query tiles) over caches
+    # of ragged lengths, several key tiles and chunks each
+    lens = [1, 130, 700, 2100, 257]
+    cpu, gpu = _small(H_I=H_I, d_I=d_I, H=16, lens=lens, lens_q=[1] * len(lens), k=64,
+                      integer=integer, seed=108)
+    g = C.np_(C.gpu_indexer(gpu))
+    C.assert_no_device_error()
+    for b in range(len(lens)):
+        q0, q1, _, _ = C.seq_slices(cpu, b)
+        o = C.oracle_scores(cpu, b)
+        bound = None if integer else C.oracle_scores(cpu, b, abs_bound=True)
+        C.check_indexer(g[q0:q1], o, bound, _p_rows(cpu, b, [0]), exact=integer)
+
+
 # --------------------------------------------------------------------------
 # Top-k (same fp32 scores on both sides -> bit-exact)
 # --------------------------------------------------------------------------
