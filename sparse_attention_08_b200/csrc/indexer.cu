@@ -263,11 +263,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* wq = wq_s + eg * kHalf;
     int64_t ac = 0;
     bool ok = true;
-    for (int64_t item = blockIdx.x; ok && item < P.n_items; item += gridDim.x) {
+    for (int64_t item = blockIdx.x; item < P.n_items; item += gridDim.x) {
       Item it;
       if (!decode_item<QPT>(item, P, it)) continue;
+      // the warpgroup stops together once a wait of one of its warps gave up
+      if (named_bar_or(bar_id, kEpiThreads, !ok)) break;
       // head weights of this half of the query group: w * q_scale
-      named_bar_sync(bar_id, kEpiThreads);
       for (int n = et; n < kHalf; n += kEpiThreads) {
         const int col = hf * kHalf + n;
         const int qi = col / H_I;

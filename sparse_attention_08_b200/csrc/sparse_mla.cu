@@ -278,11 +278,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // slot -1 is the query tile, slots 0..nb-1 the blocks
       for (int j = -1; j < it.nb; ++j, ++u) {
         const uint32_t st = u % kStages;
-        if (tg == 0 &&
-            !mbar_wait(kv_empty(st), static_cast<uint32_t>(((u / kStages) & 1) ^ 1), P.err))
-          *abort_flag = 1;
-        named_bar_sync(kBarProducer, kProdThreads);
-        if (*abort_flag) {
+        // every filler thread takes the same decision to stop
+        const bool failed =
+            tg == 0 && !mbar_wait(kv_empty(st), static_cast<uint32_t>(((u / kStages) & 1) ^ 1), P.err);
+        if (named_bar_or(kBarProducer, kProdThreads, failed || *abort_flag)) {
+          if (failed) *abort_flag = 1;
           ok = false;
           break;
         }

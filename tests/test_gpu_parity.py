@@ -170,7 +170,10 @@ def _attention_vs_oracle(cpu, gpu, idx_gpu):
                              np.concatenate(gl_all), np.concatenate(ol_all))
 
 
-@pytest.mark.parametrize("H,k", [(16, 64), (128, 100), (64, 256), (32, 130)])
+# H <= 64 runs one CTA per 64-head group; H > 64 runs CTA pairs over
+# 128-head groups (192: a second group with only 64 real heads).
+@pytest.mark.parametrize("H,k", [(16, 64), (128, 100), (64, 256), (32, 130), (192, 128),
+                                 (256, 64)])
 def test_attention_small(H, k):
     cpu, gpu = _small(H_I=8, d_I=64, H=H, lens=[400, 300], lens_q=[400, 90], k=k, seed=105)
     idx, _ = C.gpu_topk(gpu, C.gpu_indexer(gpu), with_val=False)
@@ -192,8 +195,9 @@ def test_attention_rescales_when_the_maximum_jumps():
     _attention_vs_oracle(cpu, gpu, idx)
 
 
-def test_attention_skips_invalid_entries():
-    cpu, gpu = _small(H_I=8, d_I=64, H=64, L=300, k=128, seed=107)
+@pytest.mark.parametrize("H", [64, 128])
+def test_attention_skips_invalid_entries(H):
+    cpu, gpu = _small(H_I=8, d_I=64, H=H, L=300, k=128, seed=107)
     idx, _ = C.gpu_topk(gpu, C.gpu_indexer(gpu), with_val=False)
     bad = idx.clone()
     bad[5:, 3] = -1                 # holes inside the valid prefix
