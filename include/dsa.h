@@ -192,6 +192,47 @@ DSA_API dsa_status_t dsa_forward_noalloc(const void* q_fp8, const float* q_scale
                                          int d_I, int H, int d_qk, int d_v, int k, float sm_scale,
                                          void* out, float* lse, int32_t* idx_out, void* stream);
 
+/*
+ * dsa_forward with every input and output in HOST memory: the call copies
+ * what the path needs to the GPU, runs it and copies the results back, and
+ * returns when `out` and `lse` hold them.  The method's statement (each
+ * query's scores, selection and attention read only that query's row and the
+ * key-side tensors: "DeepSeek V3.2 and the lightning indexer", section "How
+ * the lightning indexer works") lets the query rows go through in chunks of
+ * `chunk_q` rows: the key-side tensors (k_fp8, k_scale, kv) are copied once,
+ * and chunk c is uploaded, computed and downloaded on streams[c % n_streams],
+ * so copies of one chunk overlap the kernels of another.  Results are
+ * bitwise those of dsa_forward on the same inputs.
+ *
+ *  - Every pointer argument except `workspace` and `streams` is a host
+ *    pointer, with the layouts of dsa_forward; cu_seqlens_q/k are host
+ *    arrays [B+1] that start at 0 and end at total_q / total_k.  Page-locked
+ *    (pinned) host memory is needed for the copies to overlap; pageable
+ *    memory works but serialises them.
+ *  - `workspace`: device memory, 256-byte aligned, of at least
+ *    dsa_forward_host_workspace_size(total_k, max_len_k, B, H_I, d_I, H, k,
+ *    chunk_q, n_streams) bytes, owned by the caller.
+ *  - `streams`: n_streams >= 1 CUDA streams owned by the caller (streams[0]
+ *    carries the one-time key copies; the others wait for them).  The call
+ *    synchronises all of them before it returns.
+ *  - lse may be NULL.  Errors as dsa_forward, plus DSA_ERR_INVALID_ARG for
+ *    cu_seqlens that do not describe the batch.
+ */
+DSA_API dsa_status_t dsa_forward_host(const void* q_fp8, const float* q_scale, const float* w,
+                                      const void* k_fp8, const float* k_scale, const void* q,
+                                      const void* kv, const int32_t* cu_seqlens_q,
+                                      const int32_t* cu_seqlens_k, int B, int max_len_q,
+                                      int max_len_k, int64_t total_q, int64_t total_k, int H_I,
+                                      int d_I, int H, int d_qk, int d_v, int k, float sm_scale,
+                                      void* out, float* lse, int chunk_q, void* workspace,
+                                      size_t workspace_bytes, void* const* streams, int n_streams);
+
+/* Device workspace bytes for dsa_forward_host: the key-side tensors once, and
+ * per stream one chunk's query rows, outputs and dsa_forward workspace.
+ * Returns 0 for invalid sizes. */
+DSA_API size_t dsa_forward_host_workspace_size(int64_t total_k, int max_len_k, int B, int H_I,
+                                               int d_I, int H, int k, int chunk_q, int n_streams);
+
 /* Bytes of workspace dsa_forward needs: an f32 score matrix [total_q,
  * round_up(max_len_k, 4)] plus an int32 index matrix [total_q, k], each
  * 256-byte aligned.  Returns 0 for invalid sizes. */

@@ -14,7 +14,8 @@ import os
 __all__ = [
     "DSAError", "lib_path", "load", "dsa_version", "dsa_status_string",
     "dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward",
-    "dsa_forward_workspace_size", "dsa_get_device_error", "dsa_forward_noalloc", "EXPORTED",
+    "dsa_forward_workspace_size", "dsa_get_device_error", "dsa_forward_noalloc",
+    "dsa_forward_host", "dsa_forward_host_workspace_size", "EXPORTED",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -25,7 +26,7 @@ _lib = None
 EXPORTED = (
     "dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward",
     "dsa_forward_workspace_size", "dsa_status_string", "dsa_get_device_error", "dsa_version",
-    "dsa_forward_noalloc",
+    "dsa_forward_noalloc", "dsa_forward_host", "dsa_forward_host_workspace_size",
 )
 
 STATUS = {
@@ -62,8 +63,12 @@ def load():
                                 P, P, P, P, ctypes.c_size_t, P]
     lib.dsa_forward_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I64, I64, I, I, I, I,
                                         I, I, F, P, P, P, P]
+    lib.dsa_forward_host.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I64, I64, I, I, I, I, I,
+                                     I, F, P, P, I, P, ctypes.c_size_t, P, I]
+    lib.dsa_forward_host_workspace_size.argtypes = [I64, I, I, I, I, I, I, I, I]
+    lib.dsa_forward_host_workspace_size.restype = ctypes.c_size_t
     for name in ("dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward",
-                 "dsa_forward_noalloc"):
+                 "dsa_forward_noalloc", "dsa_forward_host"):
         getattr(lib, name).restype = I
     lib.dsa_forward_workspace_size.argtypes = [I64, I, I]
     lib.dsa_forward_workspace_size.restype = ctypes.c_size_t
@@ -228,6 +233,58 @@ def dsa_forward_noalloc(q_fp8, q_scale, w, k_fp8, k_scale, q, kv, cu_seqlens_q, 
                                     int(out.shape[2]), int(k), float(sm_scale), _ptr(out),
                                     _ptr(lse), _ptr(idx_out), _stream(stream))
     _check(rc, "dsa_forward_noalloc")
+
+
+def _need_host(t, dtype, name, ndim=None):
+    if t is None:
+        return
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims")
+
+
+def dsa_forward_host_workspace_size(total_k, max_len_k, B, H_I, d_I, H, k, chunk_q,
+                                    n_streams) -> int:
+    return int(load().dsa_forward_host_workspace_size(int(total_k), int(max_len_k), int(B),
+                                                      int(H_I), int(d_I), int(H), int(k),
+                                                      int(chunk_q), int(n_streams)))
+
+
+def dsa_forward_host(q_fp8, q_scale, w, k_fp8, k_scale, q, kv, cu_seqlens_q, cu_seqlens_k, B,
+                     max_len_q, max_len_k, k, sm_scale, out, lse, chunk_q, workspace, streams):
+    """dsa_forward over host tensors (pin them for the copies to overlap):
+    the library uploads the key side once and the query rows in chunks of
+    chunk_q rows spread over `streams` (torch.cuda.Stream objects), and returns
+    with `out` / `lse` (host tensors) filled.  `workspace` is a uint8 CUDA
+    tensor of dsa_forward_host_workspace_size(...) bytes."""
+    import torch
+    q8 = q_fp8.view(torch.uint8) if q_fp8.dtype == torch.float8_e4m3fn else q_fp8
+    k8 = k_fp8.view(torch.uint8) if k_fp8.dtype == torch.float8_e4m3fn else k_fp8
+    for t, dt, name, nd in ((q8, torch.uint8, "q_fp8", 3), (k8, torch.uint8, "k_fp8", 2),
+                            (q_scale, torch.float32, "q_scale", 2), (w, torch.float32, "w", 2),
+                            (k_scale, torch.float32, "k_scale", 1),
+                            (q, torch.bfloat16, "q", 3), (kv, torch.bfloat16, "kv", 2),
+                            (cu_seqlens_q, torch.int32, "cu_seqlens_q", 1),
+                            (cu_seqlens_k, torch.int32, "cu_seqlens_k", 1),
+                            (out, torch.bfloat16, "out", 3), (lse, torch.float32, "lse", 2)):
+        _need_host(t, dt, name, nd)
+    _need(workspace, torch.uint8, "workspace", 1)
+    T_q, H_I, d_I = q8.shape
+    _, H, d_qk = q.shape
+    arr = (ctypes.c_void_p * len(streams))(*[s.cuda_stream for s in streams])
+    rc = load().dsa_forward_host(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale),
+                                 _ptr(q), _ptr(kv), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+                                 int(B), int(max_len_q), int(max_len_k), int(T_q),
+                                 int(k8.shape[0]), int(H_I), int(d_I), int(H), int(d_qk),
+                                 int(out.shape[2]), int(k), float(sm_scale), _ptr(out),
+                                 _ptr(lse), int(chunk_q), _ptr(workspace),
+                                 int(workspace.numel()), arr, len(streams))
+    _check(rc, "dsa_forward_host")
 
 
 def dsa_get_device_error(stream=None) -> int:

@@ -106,6 +106,37 @@ def test_forward_workspace_checks():
     assert fwd(_fake(0x10001), need) == ALIGN
 
 
+def test_forward_host_checks_before_any_device_call():
+    """Argument checks of the host-buffer entry point run on the host: each of
+    these returns its status without touching a device."""
+    import numpy as np
+    lib = dsa.load()
+    f = ctypes.c_float(1.0 / 24)
+    cu_q = np.array([0, 64], dtype=np.int32)
+    cu_k = np.array([0, 64], dtype=np.int32)
+    bad_k = np.array([0, 32], dtype=np.int32)          # fewer keys than queries
+    p = _fake()
+    need = dsa.dsa_forward_host_workspace_size(64, 64, 1, 64, 128, 128, 16, 32, 2)
+    assert need > 0
+    # one more stream costs one more chunk region
+    assert dsa.dsa_forward_host_workspace_size(64, 64, 1, 64, 128, 128, 16, 32, 3) > need
+    assert dsa.dsa_forward_host_workspace_size(64, 64, 1, 64, 128, 128, 16, 0, 2) == 0
+    streams = (ctypes.c_void_p * 2)(_fake().value, _fake().value)
+
+    def host(cq, ck, chunk=32, ws=p, nbytes=need, st=streams, n=2, d_qk=576):
+        return lib.dsa_forward_host(p, p, p, p, p, p, p, cq.ctypes.data, ck.ctypes.data, 1, 64, 64,
+                                    64, int(ck[-1]), 64, 128, 128, d_qk, 512, 16, f, p, None,
+                                    chunk, ws, nbytes, st, n)
+    assert host(cu_q, cu_k, chunk=0) == INVALID
+    assert host(cu_q, cu_k, st=None) == INVALID
+    assert host(cu_q, cu_k, n=0) == INVALID
+    assert host(cu_q, bad_k) == INVALID
+    assert host(cu_q, cu_k, d_qk=512) == UNSUPPORTED
+    assert host(cu_q, cu_k, ws=None) == WORKSPACE
+    assert host(cu_q, cu_k, nbytes=need - 1) == WORKSPACE
+    assert host(cu_q, cu_k, ws=_fake(0x10010)) == ALIGN
+
+
 def _have_gpu():
     try:
         import torch

@@ -9,6 +9,7 @@ import pytest
 import torch
 
 import oracle
+import sparse_attention_08_b200 as dsa
 from sparse_attention_08_b200 import workloads as W
 from tests import dsa_cases as C
 
@@ -223,6 +224,33 @@ def test_forward_end_to_end_small_varlen():
         C.check_topk_near_cut(g_idx[q0:q1], o_idx, sc, _p_rows(cpu, b, rows), cpu.k)
         o, ol = C.oracle_attention(cpu, b, g_idx[q0:q1], rows)
         C.check_attention(g_out[q0:q1], o, g_lse[q0:q1], ol)
+
+
+# Host-buffer entry point: the batch goes through in chunks of query rows on
+# several streams; each row's arithmetic is unchanged, so the results are
+# bitwise those of dsa_forward.  The chunk sizes cut sequences in the middle
+# and put several sequences (one without queries) into one chunk.
+@pytest.mark.parametrize("chunk,n_streams", [(64, 3), (333, 2), (5000, 1)])
+def test_forward_host_matches_forward(chunk, n_streams):
+    cpu, gpu = _small(H_I=64, d_I=128, H=128, lens=[1100, 200, 700, 300],
+                      lens_q=[1100, 0, 1, 45], k=256, seed=111)
+    _, out_ref, lse_ref = C.gpu_forward(gpu)
+    names = ("q8", "q_scale", "w", "k8", "k_scale", "q", "kv", "cu_q", "cu_k")
+    h = {n: getattr(cpu, n).contiguous().pin_memory() for n in names}
+    H = cpu.q.shape[1]
+    out = torch.full((cpu.T_q, H, 512), float("nan"), dtype=torch.bfloat16).pin_memory()
+    lse = torch.full((cpu.T_q, H), float("nan"), dtype=torch.float32).pin_memory()
+    nbytes = dsa.dsa_forward_host_workspace_size(cpu.T_k, cpu.max_len_k, cpu.B, 64, 128, H,
+                                                 cpu.k, chunk, n_streams)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    streams = [torch.cuda.Stream() for _ in range(n_streams)]
+    torch.cuda.synchronize()
+    dsa.dsa_forward_host(h["q8"], h["q_scale"], h["w"], h["k8"], h["k_scale"], h["q"], h["kv"],
+                         h["cu_q"], h["cu_k"], cpu.B, cpu.max_len_q, cpu.max_len_k, cpu.k,
+                         cpu.scale, out, lse, chunk, ws, streams)
+    C.assert_no_device_error()
+    assert np.array_equal(C.bits(out), C.bits(out_ref.cpu()))
+    assert np.array_equal(C.np_(lse).view(np.uint32), C.np_(lse_ref).view(np.uint32))
 
 
 def test_config0_full_exact():
