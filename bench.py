@@ -355,7 +355,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-E2E_CHUNK = 2048        # query rows per chunk of the host-buffer pipeline
+E2E_CHUNK = 1024        # query rows per chunk of the host-buffer pipeline
 E2E_STREAMS = 3
 
 
