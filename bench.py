@@ -235,7 +235,11 @@ def run_ours(args):
     dsa.load()
     cfg = W.CONFIGS[args.config]
     seed = rank_seed(args.config, rank)
-    wl = W.make_prefill(args.config, device="cuda", seed=seed)
+    if cfg.decode:
+        # a varlen decode batch (not the headline; a measurement of that shape)
+        wl = W.make_decode(args.config, device="cuda", seed=seed)
+    else:
+        wl = W.make_prefill(args.config, device="cuda", seed=seed)
     H_I, d_I, H = wl.q8.shape[1], wl.q8.shape[2], wl.q.shape[1]
     ld = (wl.max_len_k + 3) // 4 * 4
     logits = torch.empty((wl.T_q, ld), dtype=torch.float32, device="cuda")
@@ -330,7 +334,7 @@ def run_ours(args):
 
     # ---- CPU baseline: the oracle, rank 0 at N=1 only
     cpu = None
-    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+    if world == 1 and rank == 0 and not args.no_cpu_baseline and not cfg.decode:
         n_rows = max(8, min(64, 2 * oracle_threads()))
         dt, desc = oracle_sample(wl, n_rows, seed=99)
         cpu = {"value": round(n_rows / dt, 4), "unit": UNIT, "cores": oracle_threads(),
@@ -342,7 +346,7 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "fp8e4m3+bf16", "data": "synthetic",
-            "config": {"workload": f"{cfg.name} (one causal prefill per GPU)", "L": cfg.L,
+            "config": {"workload": f"{cfg.name} (" + ("one varlen decode batch" if cfg.decode else "one causal prefill") + " per GPU)", "L": cfg.L,
                        "H_I": H_I, "d_I": d_I, "H": H, "d_qk": 576, "d_v": 512, "k": wl.k,
                        "global_batch_sequences": world, "parallelism": f"dp{world}",
                        "l2": "flushed between steps (256 MiB write outside the timed events)"},

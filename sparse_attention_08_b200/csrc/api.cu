@@ -142,9 +142,12 @@ dsa_status_t dsa_indexer_logits(const void* q_fp8, const float* q_scale, const f
   if ((st = device_info(&dev)) != DSA_OK) return st;
   const CUtensorMapSwizzle swz =
       d_I == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  // A tile holds 256 (query, head) columns; when every sequence has a single
+  // query (decode) and the heads fit, one query of 64 columns instead.
+  const int tile_n = (max_len_q <= 1 && H_I >= 16 && H_I <= 64) ? 64 : 256;
   CUtensorMap tq, tk;
-  if ((st = encode_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_fp8, total_q * H_I, d_I, 1, 256, d_I,
-                      swz)) != DSA_OK)
+  if ((st = encode_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_fp8, total_q * H_I, d_I, 1,
+                      static_cast<uint32_t>(tile_n), d_I, swz)) != DSA_OK)
     return st;
   if ((st = encode_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, k_fp8, total_k, d_I, 1, 128, d_I,
                       swz)) != DSA_OK)
@@ -162,6 +165,7 @@ dsa_status_t dsa_indexer_logits(const void* q_fp8, const float* q_scale, const f
   a.d_I = d_I;
   a.logits = logits;
   a.ld = ld_logits;
+  a.tile_n = tile_n;
   return from_cuda(dsa::launch_indexer(tq, tk, a, dev->num_sms, next_err(dev),
                                        static_cast<cudaStream_t>(stream)));
 }

@@ -40,13 +40,9 @@ namespace dsa {
 namespace {
 
 constexpr int kBlockK = 128;      // keys per tile (MMA M)
-constexpr int kN = 256;           // MMA N = queries per tile * H_I
 constexpr int kKbPerItem = 16;    // key blocks per work item
 constexpr int kStages = 6;        // key-tile pipeline depth
-constexpr int kEpiGroups = 4;
 constexpr int kEpiThreads = 128;   // one epilogue warpgroup
-constexpr int kThreads = 64 + kEpiGroups * kEpiThreads;   // producer, MMA, epilogue
-constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
 
 struct Params {
   const float* q_scale;
@@ -98,17 +94,31 @@ __device__ __forceinline__ bool decode_item(int64_t item, const Params& P, Item&
   return true;
 }
 
-template <int H_I, int D_I>
+// NT = MMA N = queries per tile * H_I: 256 (four queries of 64 heads) for
+// prefill; 64 (one query of 64 heads) when every sequence has one query
+// (decode), so a tile does not carry three empty queries.
+template <int H_I, int D_I, int NT>
 struct Layout {
-  static constexpr int QPT = kN / H_I;
-  static constexpr uint32_t kQBytes = kN * D_I;          // one query group tile
+  static constexpr int kN = NT;
+  static constexpr int QPT = NT / H_I;
+  // epilogue warpgroups per accumulator buffer: two column halves when a
+  // tile holds two or more queries, else one warpgroup reads all columns
+  static constexpr int kHalves = QPT >= 2 ? 2 : 1;
+  // accumulator buffers in TMEM: two of 256 columns fill it; 64-column tiles
+  // keep four in flight, which hides more of a tile's hand-over latency
+  static constexpr int kBufs = (NT <= 64 && kHalves == 1) ? 4 : 2;
+  static constexpr int kEpiGroups = kBufs * kHalves;
+  static constexpr int kThreads = 64 + kEpiGroups * kEpiThreads;   // producer, MMA, epilogue
+  static constexpr uint32_t kTmemCols =
+      kBufs * NT >= 512 ? 512 : (kBufs * NT >= 256 ? 256 : (kBufs * NT >= 128 ? 128 : 64));
+  static constexpr uint32_t kQBytes = NT * D_I;          // one query group tile
   static constexpr uint32_t kKBytes = kBlockK * D_I;     // one key tile
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffK = kOffQ + 2 * kQBytes;
   static constexpr uint32_t kOffWq = kOffK + kStages * kKBytes;
-  static constexpr uint32_t kOffBar = kOffWq + kEpiGroups * (kN / 2) * 4;  // wq half per warpgroup
-  // barriers: q_full[2], q_empty[2], k_full[S], k_empty[S], acc_full[2], acc_empty[2], drain
-  static constexpr uint32_t kNumBars = 2 + 2 + kStages + kStages + 2 + 2 + 1;
+  static constexpr uint32_t kOffBar = kOffWq + kEpiGroups * (kN / kHalves) * 4;  // wq per warpgroup
+  // barriers: q_full[2], q_empty[2], k_full[S], k_empty[S], acc_full[B], acc_empty[B], drain
+  static constexpr uint32_t kNumBars = 2 + 2 + kStages + kStages + 2 * kBufs + 1;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kBytes = kOffMisc + 16;
   static constexpr uint32_t kSmem = kBytes + 1024;      // + alignment slack
@@ -117,11 +127,12 @@ struct Layout {
   static constexpr uint32_t kIdesc = instr_desc(kFmtE4M3, kFmtE4M3, 0, 0, kBlockK, kN);
 };
 
-template <int H_I, int D_I>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int H_I, int D_I, int NT>
+__global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_k, const Params P) {
-  using L = Layout<H_I, D_I>;
+  using L = Layout<H_I, D_I, NT>;
+  constexpr int kN = L::kN;
   constexpr int QPT = L::QPT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -133,9 +144,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto q_empty = [&](int i) { return bar0 + 8u * (2 + i); };
   auto k_full = [&](int i) { return bar0 + 8u * (4 + i); };
   auto k_empty = [&](int i) { return bar0 + 8u * (4 + kStages + i); };
+  constexpr int kBufs = L::kBufs;
   auto acc_full = [&](int i) { return bar0 + 8u * (4 + 2 * kStages + i); };
-  auto acc_empty = [&](int i) { return bar0 + 8u * (6 + 2 * kStages + i); };
-  const uint32_t drain_bar = bar0 + 8u * (8 + 2 * kStages);
+  auto acc_empty = [&](int i) { return bar0 + 8u * (4 + 2 * kStages + kBufs + i); };
+  const uint32_t drain_bar = bar0 + 8u * (4 + 2 * kStages + 2 * kBufs);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
 
@@ -146,8 +158,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(q_full(i), 1);
       mbar_init(q_empty(i), 1);
+    }
+    for (int i = 0; i < kBufs; ++i) {
       mbar_init(acc_full(i), 1);
-      mbar_init(acc_empty(i), 8);     // every warp of both column halves reads the buffer
+      mbar_init(acc_empty(i), 4 * L::kHalves);   // every warp that reads the buffer
     }
     for (int i = 0; i < kStages; ++i) {
       mbar_init(k_full(i), 1);
@@ -160,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmap_k);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), kTmemCols);
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), L::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -215,8 +229,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < it.nkb; ++j) {
           const int st = static_cast<int>(kc % kStages);
           if (!(ok = mbar_wait(k_full(st), static_cast<uint32_t>((kc / kStages) & 1), P.err))) break;
-          const int ab = static_cast<int>(ac & 1);
-          if (!(ok = mbar_wait(acc_empty(ab), static_cast<uint32_t>(((ac >> 1) & 1) ^ 1), P.err)))
+          const int ab = static_cast<int>(ac % kBufs);
+          if (!(ok = mbar_wait(acc_empty(ab), static_cast<uint32_t>(((ac / kBufs) & 1) ^ 1), P.err)))
             break;
           tc_fence_after();
           const uint32_t k_addr = sbase + L::kOffK + st * L::kKBytes;
@@ -243,19 +257,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // Warpgroup eg reads accumulator buffer eg/2 (every other tile) and the
-    // column half eg%2.  Warp w reads TMEM lanes 32*(w%4)..; a thread owns
-    // one key of the tile.
+    // Warpgroup eg reads accumulator buffer eg / kHalves (every kBufs-th
+    // tile) and the column half eg % kHalves.  Warp w reads TMEM lanes
+    // 32*(w%4)..; a thread owns one key of the tile.
     const int eg = (warp - 2) >> 2;            // warpgroup 0..3
-    const int ab_mine = eg >> 1;
-    const int hf = eg & 1;
+    const int ab_mine = eg / L::kHalves;
+    const int hf = eg % L::kHalves;
     const int et = threadIdx.x - 64 - eg * kEpiThreads;   // 0..127 within the group
     const uint32_t bar_id = 1 + eg;
     const int sp = warp & 3;                  // TMEM sub-partition of this warp
     const int row = sp * 32 + lane;           // TMEM lane = key within the tile
     const uint32_t lane_addr = static_cast<uint32_t>(sp * 32) << 16;
-    constexpr int kHalf = kN / 2;             // columns per warpgroup
-    constexpr int QH = QPT / 2;               // queries per warpgroup
+    constexpr int kHalf = kN / L::kHalves;    // columns per warpgroup
+    constexpr int QH = QPT / L::kHalves;      // queries per warpgroup
     // independent FMA chains per query (latency hiding)
     constexpr int NCH = H_I >= 16 ? 4 : (H_I >= 8 ? 2 : 1);
     // chunks of 32 columns loaded per tcgen05.wait (register budget)
@@ -281,10 +295,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       named_bar_sync(bar_id, kEpiThreads);
       for (int j = 0; j < it.nkb; ++j, ++ac) {
-        const int ab = static_cast<int>(ac & 1);
+        const int ab = static_cast<int>(ac % kBufs);
         if (ab != ab_mine) continue;
         // each warp waits and releases on its own: no warpgroup barrier per tile
-        if (!warp_wait(acc_full(ab), static_cast<uint32_t>((ac >> 1) & 1), P.err)) {
+        if (!warp_wait(acc_full(ab), static_cast<uint32_t>((ac / kBufs) & 1), P.err)) {
           *abort_flag = 1;
           ok = false;
           break;
@@ -346,14 +360,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, L::kTmemCols);
   }
 }
 
-template <int H_I, int D_I>
+template <int H_I, int D_I, int NT>
 cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const IndexerArgs& a,
                      int num_sms, DevErr err, cudaStream_t s) {
-  using L = Layout<H_I, D_I>;
+  using L = Layout<H_I, D_I, NT>;
   Params P;
   P.q_scale = a.q_scale;
   P.w = a.w;
@@ -382,11 +396,11 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const Indexer
   };
   while (gcd(P.n_kc, grid) != 1) ++P.n_kc;
   P.n_items = static_cast<int64_t>(a.B) * P.n_qg * P.n_kc;
-  auto kern = indexer_kernel<H_I, D_I>;
+  auto kern = indexer_kernel<H_I, D_I, NT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(L::kSmem));
   if (e != cudaSuccess) return e;
-  kern<<<static_cast<unsigned>(grid), kThreads, L::kSmem, s>>>(tq, tk, P);
+  kern<<<static_cast<unsigned>(grid), L::kThreads, L::kSmem, s>>>(tq, tk, P);
   return cudaGetLastError();
 }
 
@@ -394,8 +408,10 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const Indexer
 
 cudaError_t launch_indexer(const CUtensorMap& tq, const CUtensorMap& tk, const IndexerArgs& a,
                            int num_sms, DevErr err, cudaStream_t s) {
-#define DSA_IDX_CASE(h, d) \
-  if (a.H_I == h && a.d_I == d) return launch_t<h, d>(tq, tk, a, num_sms, err, s);
+#define DSA_IDX_CASE(h, d)                                                               \
+  if (a.H_I == h && a.d_I == d && a.tile_n == 256) return launch_t<h, d, 256>(tq, tk, a, num_sms, err, s);
+#define DSA_IDX_CASE_DECODE(h, d)                                                        \
+  if (a.H_I == h && a.d_I == d && a.tile_n == 64) return launch_t<h, d, 64>(tq, tk, a, num_sms, err, s);
   DSA_IDX_CASE(4, 64)
   DSA_IDX_CASE(8, 64)
   DSA_IDX_CASE(16, 64)
@@ -408,7 +424,14 @@ cudaError_t launch_indexer(const CUtensorMap& tq, const CUtensorMap& tk, const I
   DSA_IDX_CASE(32, 128)
   DSA_IDX_CASE(64, 128)
   DSA_IDX_CASE(128, 128)
+  DSA_IDX_CASE_DECODE(16, 64)
+  DSA_IDX_CASE_DECODE(32, 64)
+  DSA_IDX_CASE_DECODE(64, 64)
+  DSA_IDX_CASE_DECODE(16, 128)
+  DSA_IDX_CASE_DECODE(32, 128)
+  DSA_IDX_CASE_DECODE(64, 128)
 #undef DSA_IDX_CASE
+#undef DSA_IDX_CASE_DECODE
   return cudaErrorInvalidValue;
 }
 

@@ -20,6 +20,7 @@ struct IndexerArgs {
   int H_I, d_I;
   float* logits;
   int64_t ld;
+  int tile_n;   // MMA N of a tile: 256 (four queries x 64 heads) or 64 (decode)
 };
 
 struct TopkArgs {
