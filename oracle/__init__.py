@@ -70,6 +70,9 @@ def _load():
         lib.oracle_sparse_mla_at.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, i32,
                                              ctypes.c_double, P, P]
         lib.oracle_num_threads.restype = i32
+        lib.oracle_indexer_kl_at.argtypes = [P, P, P, P, P, i64, i64, i64, i32, i32, i32,
+                                             ctypes.c_double, P, P, P]
+        lib.oracle_indexer_kl_at.restype = i32
         lib.oracle_num_threads.argtypes = []
         _lib = lib
     return _lib
@@ -245,3 +248,31 @@ def sparse_mla_at(q_bits, kv_bits, idx, pos, scale, d_v=512):
     if rc != 0:
         raise ValueError("oracle_sparse_mla_at: bad arguments")
     return out, lse
+
+
+def indexer_kl_at(q_bits, kv_bits, idx, pos, logits, scale):
+    """KL alignment of the indexer to the main attention over each row's
+    selection ("DeepSeek V3.2 and the lightning indexer", "Teaching a dense
+    model to be sparse"; "DeepSeek-V3.2" atlas entry, "Design overview"): row r
+    (query at position pos[r], index row idx[r], indexer scores logits[r, :])
+    gets the target p = head-averaged attention distribution over its valid
+    selected entries, the loss KL(p || softmax(I)) and the gradient
+    softmax(I) - p.  Returns (kl [R], grad [R, k], target [R, k]) in fp64, the
+    last two in index-row order with zeros at invalid entries."""
+    q_bits = _c(q_bits, np.uint16)
+    kv_bits = _c(kv_bits, np.uint16)
+    idx = _c(idx, np.int32)
+    pos = _c(pos, np.int64)
+    logits = _c(logits, np.float32)
+    R, H, d_qk = q_bits.shape
+    n_k = kv_bits.shape[0]
+    k = idx.shape[1]
+    kl = np.empty((R,), dtype=np.float64)
+    grad = np.empty((R, k), dtype=np.float64)
+    target = np.empty((R, k), dtype=np.float64)
+    rc = _load().oracle_indexer_kl_at(_ptr(q_bits), _ptr(kv_bits), _ptr(idx), _ptr(pos),
+                                      _ptr(logits), int(logits.shape[1]), R, n_k, H, d_qk, k,
+                                      float(scale), _ptr(kl), _ptr(grad), _ptr(target))
+    if rc != 0:
+        raise ValueError("oracle_indexer_kl_at: bad arguments")
+    return kl, grad, target

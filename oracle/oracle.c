@@ -37,7 +37,10 @@
  *  - top-k: the min(k, p+1) largest scores, ties to the lower index, -0 equal
  *    to +0, emitted in ascending index order and padded with -1;
  *  - attention: o[t,h] = sum_s softmax_s(scale * q[t,h,:] . c[s,:]) * c[s,0:d_v]
- *    over the selected set, lse = log sum_s exp(scale * q . c).
+ *    over the selected set, lse = log sum_s exp(scale * q . c);
+ *  - indexer training signal (oracle_indexer_kl_at): target p = the head
+ *    average of the attention distributions over the selected set, loss
+ *    KL(p || softmax(I)) over that set, gradient softmax(I) - p.
  *
  * Parity pins: tests/test_oracle_pins.py checks every function here against
  * brute force, closed forms, invariants and library routines.
@@ -398,6 +401,104 @@ int oracle_sparse_mla_at(const uint16_t* q, const uint16_t* kv, const int32_t* i
     }
     free(sel);
     free(x);
+  }
+  return bad ? -1 : 0;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Indexer training signal.                                                 */
+/* ---------------------------------------------------------------------- */
+
+/* KL alignment of the indexer to the main attention over the selected set
+ * ("DeepSeek V3.2 and the lightning indexer", section "Teaching a dense model
+ * to be sparse": the indexer is trained with a KL divergence loss to match
+ * the distribution of the main attention; "DeepSeek-V3.2" atlas entry,
+ * "Design overview": the target is the head-wise attention distribution
+ * summed over heads).  Readings: the target of query row r over its valid
+ * selected entries S (the index row's entries 0 <= s <= p) is
+ *     p[s] = (1/H) sum_h softmax_{s in S}(scale * q[r,h,:] . c[s,:]),
+ * the indexer's distribution is q[s] = softmax_{s in S}(I[r, s]) of the given
+ * scores, the loss is KL(p || q) = sum_s p[s] (log p[s] - log q[s]) and the
+ * gradient of the loss with respect to I[r, s] is q[s] - p[s].
+ * Row r of q is at position pos[r]; its scores are logits[r * ld + s].
+ * Outputs per row: kl[r]; grad and target (nullable) n_rows x k in index-row
+ * order, 0 at invalid entries.  The attention scores are taken afresh in fp64
+ * (this function does not use the attention's lse). */
+int oracle_indexer_kl_at(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
+                         const int64_t* pos, const float* logits, int64_t ld, int64_t n_rows,
+                         int64_t n_k, int H, int d_qk, int k, double scale, double* kl,
+                         double* grad, double* target) {
+  if (k <= 0 || H <= 0 || !pos || !logits || !kl) return -1;
+  int bad = 0;
+#pragma omp parallel
+  {
+    int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+    int32_t* slot = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+    double* x = (double*)malloc(sizeof(double) * (size_t)k);
+    double* pt = (double*)malloc(sizeof(double) * (size_t)k);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; ++r) {
+      const int64_t p = pos[r];
+      if (p < 0 || p >= n_k || !sel || !slot || !x || !pt) {
+        bad = 1;
+        continue;
+      }
+      const int32_t* row = idx + r * (int64_t)k;
+      int64_t n = 0;
+      for (int j = 0; j < k; ++j)
+        if (row[j] >= 0 && row[j] <= p) {
+          sel[n] = row[j];
+          slot[n] = j;
+          ++n;
+        }
+      double* g = grad ? grad + r * (int64_t)k : NULL;
+      double* tg = target ? target + r * (int64_t)k : NULL;
+      for (int j = 0; j < k; ++j) {
+        if (g) g[j] = 0.0;
+        if (tg) tg[j] = 0.0;
+      }
+      if (n == 0) {
+        kl[r] = 0.0;
+        continue;
+      }
+      /* target: each head's softmax over S, averaged over the heads */
+      for (int64_t e = 0; e < n; ++e) pt[e] = 0.0;
+      for (int h = 0; h < H; ++h) {
+        const uint16_t* qh = q + (r * H + h) * (int64_t)d_qk;
+        double m = -INFINITY;
+        for (int64_t e = 0; e < n; ++e) {
+          const uint16_t* c = kv + (int64_t)sel[e] * d_qk;
+          double dot = 0.0;
+          for (int d = 0; d < d_qk; ++d) dot += oracle_bf16_decode(qh[d]) * oracle_bf16_decode(c[d]);
+          x[e] = scale * dot;
+          if (x[e] > m) m = x[e];
+        }
+        double z = 0.0;
+        for (int64_t e = 0; e < n; ++e) z += exp(x[e] - m);
+        for (int64_t e = 0; e < n; ++e) pt[e] += exp(x[e] - m) / z / (double)H;
+      }
+      /* the indexer's distribution: softmax of its scores over S */
+      double mi = -INFINITY;
+      for (int64_t e = 0; e < n; ++e) {
+        x[e] = (double)logits[r * ld + sel[e]];
+        if (x[e] > mi) mi = x[e];
+      }
+      double zi = 0.0;
+      for (int64_t e = 0; e < n; ++e) zi += exp(x[e] - mi);
+      const double log_zi = log(zi);
+      double loss = 0.0;
+      for (int64_t e = 0; e < n; ++e) {
+        const double log_q = x[e] - mi - log_zi;
+        if (pt[e] > 0.0) loss += pt[e] * (log(pt[e]) - log_q);
+        if (g) g[slot[e]] = exp(log_q) - pt[e];
+        if (tg) tg[slot[e]] = pt[e];
+      }
+      kl[r] = loss;
+    }
+    free(sel);
+    free(slot);
+    free(x);
+    free(pt);
   }
   return bad ? -1 : 0;
 }

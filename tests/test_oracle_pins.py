@@ -340,3 +340,107 @@ def test_position_explicit_entries_match_row_entries():
     assert np.array_equal(idx, i2) and np.array_equal(out, o2) and np.array_equal(lse, l2)
     o3, l3 = oracle.sparse_mla_at(qb[rows], kvb, idx, rows, wl.scale)
     assert np.array_equal(out, o3) and np.array_equal(lse, l3)
+
+
+# --------------------------------------------------------------------------
+# Indexer training signal: KL(head-averaged attention || softmax of the
+# indexer scores) over the selection ("DeepSeek V3.2 and the lightning
+# indexer", "Teaching a dense model to be sparse"; "DeepSeek-V3.2" atlas
+# entry, "Design overview").
+# --------------------------------------------------------------------------
+
+def _kl_case(R=4, H=4, n_k=60, k=24, seed=11, q_div=24.0, holes=True):
+    g = torch.Generator().manual_seed(seed)
+    rng = np.random.default_rng(seed)
+    q = (torch.randn(R, H, 576, generator=g) / q_div).to(torch.bfloat16)
+    kv = torch.randn(n_k, 576, generator=g).to(torch.bfloat16)
+    pos = np.arange(n_k - R, n_k, dtype=np.int64)
+    idx = np.full((R, k), -1, dtype=np.int32)
+    for r in range(R):
+        sel = np.sort(rng.choice(int(pos[r]) + 1, size=min(k, int(pos[r]) + 1), replace=False))
+        idx[r, :len(sel)] = sel
+    if holes:
+        idx[0, 3] = -1                       # a hole inside the prefix
+        idx[1, 5] = int(pos[1]) + 7          # beyond p: not a valid entry
+    logits = rng.standard_normal((R, n_k)).astype(np.float32) * 2.0
+    return q, kv, idx, pos, logits
+
+
+def _valid(idx, pos):
+    return (idx >= 0) & (idx <= pos[:, None])
+
+
+def test_kl_distributions_normalised_and_gradient_sums_to_zero():
+    q, kv, idx, pos, logits = _kl_case()
+    kl, grad, target = oracle.indexer_kl_at(_bits(q), _bits(kv), idx, pos, logits, 1 / 24)
+    v = _valid(idx, pos)
+    assert np.allclose(target.sum(1), 1.0, atol=1e-12)      # p sums to 1 over S
+    assert np.allclose(grad.sum(1), 0.0, atol=1e-12)        # sum(q) - sum(p) = 0
+    assert np.all(target[~v] == 0) and np.all(grad[~v] == 0)
+    assert np.all(kl >= -1e-15)                             # Gibbs' inequality
+
+
+def test_kl_vanishes_when_the_indexer_matches_the_target():
+    q, kv, idx, pos, logits = _kl_case()
+    _, _, target = oracle.indexer_kl_at(_bits(q), _bits(kv), idx, pos, logits, 1 / 24)
+    # indexer scores = log of the target plus a per-row constant
+    lg = np.full_like(logits, -50.0)
+    for r in range(len(pos)):
+        for j in range(idx.shape[1]):
+            if target[r, j] > 0:
+                lg[r, idx[r, j]] = np.log(target[r, j]) + 3.0 * r
+    kl, grad, _ = oracle.indexer_kl_at(_bits(q), _bits(kv), idx, pos, lg.astype(np.float32),
+                                       1 / 24)
+    # float32 rounding of the scores only
+    assert np.all(np.abs(kl) < 1e-12) and np.abs(grad).max() < 1e-6
+
+
+def test_kl_two_keys_closed_form():
+    # a zero query: every head's attention is uniform over the two keys, so
+    # p = (1/2, 1/2); scores (a, 0) give q = (sigma(a), 1 - sigma(a))
+    n_k, a = 5, 1.7
+    q = torch.zeros(1, 3, 576).to(torch.bfloat16)
+    kv = torch.randn(n_k, 576, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    idx = np.array([[1, 3, -1, -1]], dtype=np.int32)
+    pos = np.array([4], dtype=np.int64)
+    logits = np.zeros((1, n_k), dtype=np.float32)
+    logits[0, 1] = a
+    kl, grad, target = oracle.indexer_kl_at(_bits(q), _bits(kv), idx, pos, logits, 1 / 24)
+    s = 1.0 / (1.0 + math.exp(-float(np.float32(a))))
+    want = 0.5 * math.log(0.5 / s) + 0.5 * math.log(0.5 / (1.0 - s))
+    assert abs(kl[0] - want) < 1e-14
+    assert np.allclose(target[0], [0.5, 0.5, 0, 0], atol=1e-15)
+    assert np.allclose(grad[0], [s - 0.5, 0.5 - s, 0, 0], atol=1e-15)
+
+
+def test_kl_gradient_matches_finite_differences():
+    q, kv, idx, pos, logits = _kl_case(R=2, seed=12)
+    kl, grad, _ = oracle.indexer_kl_at(_bits(q), _bits(kv), idx, pos, logits, 1 / 24)
+    eps = 1e-3                       # representable steps of the float32 scores
+    for r, j in [(0, 0), (0, 7), (1, 2), (1, 11)]:
+        s = idx[r, j]
+        if s < 0 or s > pos[r]:
+            continue
+        up, dn = logits.copy(), logits.copy()
+        up[r, s] += eps
+        dn[r, s] -= eps
+        d = (up[r, s] - dn[r, s]).astype(np.float64)
+        kl_up, _, _ = oracle.indexer_kl_at(_bits(q), _bits(kv), idx, pos, up, 1 / 24)
+        kl_dn, _, _ = oracle.indexer_kl_at(_bits(q), _bits(kv), idx, pos, dn, 1 / 24)
+        fd = (kl_up[r] - kl_dn[r]) / d
+        assert abs(fd - grad[r, j]) < 1e-6, (r, j, fd, grad[r, j])
+
+
+def test_kl_target_is_the_mean_of_the_single_head_targets_and_matches_attention():
+    q, kv, idx, pos, logits = _kl_case(R=3, H=5, seed=13, q_div=2.0)
+    _, _, target = oracle.indexer_kl_at(_bits(q), _bits(kv), idx, pos, logits, 1 / 24)
+    heads = [oracle.indexer_kl_at(_bits(q[:, h:h + 1]), _bits(kv), idx, pos, logits, 1 / 24)[2]
+             for h in range(q.shape[1])]
+    assert np.allclose(target, np.mean(heads, axis=0), atol=1e-14)
+    # a single head's target weights the values like that head's attention
+    out, _ = oracle.sparse_mla_at(_bits(q[:, :1]), _bits(kv), idx, pos, 1 / 24)
+    vals = kv.to(torch.float64).numpy()[:, :512]
+    for r in range(len(pos)):
+        mix = sum(heads[0][r, j] * vals[idx[r, j]] for j in range(idx.shape[1])
+                  if heads[0][r, j] > 0)
+        assert np.allclose(mix, out[r, 0], atol=1e-12)
