@@ -56,6 +56,7 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-kl", action="store_true")
     return ap.parse_args()
 
 
@@ -327,6 +328,38 @@ def run_ours(args):
                               "unit": per[n][3], "frac": round(per[n][1] / per[n][2], 4)}
                           for i, n in enumerate(names)}
 
+    # ---- the indexer's KL training signal on the same workload (not part of
+    # the step): its score products are the attention's S half, M = 128
+    kl_extra = None
+    if not args.no_kl and world == 1:
+        kl = torch.empty((wl.T_q,), dtype=torch.float32, device="cuda")
+        grad = torch.empty((wl.T_q, wl.k), dtype=torch.float32, device="cuda")
+        ws_kl = torch.empty(max(16, dsa.dsa_indexer_kl_workspace_size(wl.T_q, H, wl.k)),
+                            dtype=torch.uint8, device="cuda")
+
+        def kl_call():
+            dsa.dsa_indexer_kl(wl.q, wl.kv, idx, lse, logits, wl.cu_q, wl.cu_k, wl.B,
+                               wl.max_len_q, wl.max_len_k, wl.k, wl.scale, kl, grad,
+                               workspace=ws_kl, ld_logits=ld, stream=stream)
+        for _ in range(2):
+            kl_call()
+        kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(3)]
+        for e in kev:
+            flush.fill_(2.0)
+            e[0].record(stream)
+            kl_call()
+            e[1].record(stream)
+        torch.cuda.synchronize()
+        if dsa.dsa_get_device_error() != 0:
+            raise RuntimeError("device error in the KL measurement")
+        kl_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in kev]))
+        s_flops = c["attended_pairs"] * H * 2 * 576
+        kl_extra = {"ms": round(kl_ms, 4), "bound": "tensor",
+                    "achieved": round(s_flops / (kl_ms / 1e3) / 1e12, 2), "peak": bf16_peak,
+                    "unit": "TFLOP/s", "frac": round(s_flops / (kl_ms / 1e3) / 1e12 / bf16_peak, 4),
+                    "work": "S = Q K^T of every head and selected entry (2*576 flops each)"}
+        del ws_kl, grad
+
     # ---- end to end through dsa_forward with host buffers
     e2e = None
     if not args.no_e2e and args.e2e_steps > 0:
@@ -352,6 +385,7 @@ def run_ours(args):
                        "l2": "flushed between steps (256 MiB write outside the timed events)"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": 3 * args.steps, "clocks": clk,
+            "indexer_kl": kl_extra,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -233,6 +233,43 @@ DSA_API dsa_status_t dsa_forward_host(const void* q_fp8, const float* q_scale, c
 DSA_API size_t dsa_forward_host_workspace_size(int64_t total_k, int max_len_k, int B, int H_I,
                                                int d_I, int H, int k, int chunk_q, int n_streams);
 
+/*
+ * The indexer's training signal ("DeepSeek V3.2 and the lightning indexer",
+ * section "Teaching a dense model to be sparse": the indexer is trained with a
+ * KL divergence loss to match the distribution of the main attention;
+ * "DeepSeek-V3.2" atlas entry, "Design overview": the target is the head-wise
+ * attention distribution summed over heads).  For each query row t with valid
+ * selected entries S (idx[t, j] with 0 <= idx <= p, j < min(k, p+1)):
+ *   target p[t,s] = (1/H) sum_h exp(sm_scale * q[t,h,:] . kv[s,:] - lse[t,h]),
+ *   q_I[t,s]      = softmax over S of logits[t, s],
+ *   kl_out[t]     = sum_{s in S} p (log p - log q_I),
+ *   grad_out[t,j] = q_I[t,s] - p[t,s]  (the gradient of kl_out[t] with respect
+ *                   to logits[t,s], s = idx[t,j]); 0 at invalid entries,
+ *   target_out[t,j] = p[t,s]; 0 at invalid entries.
+ * Over all causal keys (k >= every p+1) this is the dense warm-up's loss.
+ *  - q [total_q, H, d_qk] bf16 and kv [total_k, d_qk] bf16 as for
+ *    dsa_sparse_mla_fwd (d_qk = 576); idx [total_q, k] int32 as dsa_topk
+ *    writes it; lse [total_q, H] f32, natural-log log-sum-exp of each head's
+ *    attention scores over the selection (dsa_sparse_mla_fwd's lse output);
+ *    logits [total_q, ld_logits] f32 indexer scores, row = query, column =
+ *    sequence-local key (dsa_indexer_logits' output).
+ *  - kl_out [total_q] f32; grad_out and target_out [total_q, k] f32, nullable.
+ *  - workspace: device memory of dsa_indexer_kl_workspace_size(total_q, H, k)
+ *    bytes, 16-byte aligned, owned by the caller.
+ * Errors as dsa_sparse_mla_fwd.
+ */
+DSA_API dsa_status_t dsa_indexer_kl(const void* q, const void* kv, const int32_t* idx,
+                                    const float* lse, const float* logits, int64_t ld_logits,
+                                    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                    int B, int max_len_q, int max_len_k, int64_t total_q,
+                                    int64_t total_k, int H, int d_qk, int k, float sm_scale,
+                                    float* kl_out, float* grad_out, float* target_out,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* Device workspace bytes for dsa_indexer_kl: four partial-sum slices of
+ * [total_q, k] f32 per group of 128 heads.  Returns 0 for invalid sizes. */
+DSA_API size_t dsa_indexer_kl_workspace_size(int64_t total_q, int H, int k);
+
 /* Bytes of workspace dsa_forward needs: an f32 score matrix [total_q,
  * round_up(max_len_k, 4)] plus an int32 index matrix [total_q, k], each
  * 256-byte aligned.  Returns 0 for invalid sizes. */

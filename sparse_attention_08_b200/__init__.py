@@ -15,7 +15,8 @@ __all__ = [
     "DSAError", "lib_path", "load", "dsa_version", "dsa_status_string",
     "dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward",
     "dsa_forward_workspace_size", "dsa_get_device_error", "dsa_forward_noalloc",
-    "dsa_forward_host", "dsa_forward_host_workspace_size", "EXPORTED",
+    "dsa_forward_host", "dsa_forward_host_workspace_size", "dsa_indexer_kl",
+    "dsa_indexer_kl_workspace_size", "EXPORTED",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -27,6 +28,7 @@ EXPORTED = (
     "dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward",
     "dsa_forward_workspace_size", "dsa_status_string", "dsa_get_device_error", "dsa_version",
     "dsa_forward_noalloc", "dsa_forward_host", "dsa_forward_host_workspace_size",
+    "dsa_indexer_kl", "dsa_indexer_kl_workspace_size",
 )
 
 STATUS = {
@@ -65,6 +67,11 @@ def load():
                                         I, I, F, P, P, P, P]
     lib.dsa_forward_host.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I64, I64, I, I, I, I, I,
                                      I, F, P, P, I, P, ctypes.c_size_t, P, I]
+    lib.dsa_indexer_kl.argtypes = [P, P, P, P, P, I64, P, P, I, I, I, I64, I64, I, I, I, F, P, P,
+                                   P, P, ctypes.c_size_t, P]
+    lib.dsa_indexer_kl.restype = I
+    lib.dsa_indexer_kl_workspace_size.argtypes = [I64, I, I]
+    lib.dsa_indexer_kl_workspace_size.restype = ctypes.c_size_t
     lib.dsa_forward_host_workspace_size.argtypes = [I64, I, I, I, I, I, I, I, I]
     lib.dsa_forward_host_workspace_size.restype = ctypes.c_size_t
     for name in ("dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward",
@@ -285,6 +292,40 @@ def dsa_forward_host(q_fp8, q_scale, w, k_fp8, k_scale, q, kv, cu_seqlens_q, cu_
                                  _ptr(lse), int(chunk_q), _ptr(workspace),
                                  int(workspace.numel()), arr, len(streams))
     _check(rc, "dsa_forward_host")
+
+
+def dsa_indexer_kl_workspace_size(total_q, H, k) -> int:
+    return int(load().dsa_indexer_kl_workspace_size(int(total_q), int(H), int(k)))
+
+
+def dsa_indexer_kl(q, kv, idx, lse, logits, cu_seqlens_q, cu_seqlens_k, B, max_len_q, max_len_k,
+                   k, sm_scale, kl_out, grad_out=None, target_out=None, workspace=None,
+                   ld_logits=None, stream=None):
+    """The indexer's KL training signal over each query's selection (see
+    include/dsa.h): kl_out [T_q], and optionally the gradient with respect to
+    the selected indexer scores and the head-averaged attention target, both
+    [T_q, k] in index-row order.  `workspace` (uint8 CUDA tensor) is allocated
+    here when not given."""
+    import torch
+    _need(q, torch.bfloat16, "q", 3)
+    _need(kv, torch.bfloat16, "kv", 2)
+    _need(idx, torch.int32, "idx", 2)
+    _need(lse, torch.float32, "lse", 2)
+    _need(kl_out, torch.float32, "kl_out", 1)
+    _need(grad_out, torch.float32, "grad_out", 2)
+    _need(target_out, torch.float32, "target_out", 2)
+    T_q, H, d_qk = q.shape
+    nbytes = dsa_indexer_kl_workspace_size(T_q, H, k)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    ld = logits.stride(0) if ld_logits is None else ld_logits
+    rc = load().dsa_indexer_kl(_ptr(q), _ptr(kv), _ptr(idx), _ptr(lse), _ptr(logits), int(ld),
+                               _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(B), int(max_len_q),
+                               int(max_len_k), int(T_q), int(kv.shape[0]), int(H), int(d_qk),
+                               int(k), float(sm_scale), _ptr(kl_out), _ptr(grad_out),
+                               _ptr(target_out), _ptr(workspace), int(workspace.numel()),
+                               _stream(stream))
+    _check(rc, "dsa_indexer_kl")
 
 
 def dsa_get_device_error(stream=None) -> int:

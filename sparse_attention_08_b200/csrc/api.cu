@@ -244,6 +244,58 @@ dsa_status_t dsa_sparse_mla_fwd(const void* q, const void* kv, const int32_t* id
       dsa::launch_sparse_mla(q, kv, a, next_err(dev), static_cast<cudaStream_t>(stream)));
 }
 
+size_t dsa_indexer_kl_workspace_size(int64_t total_q, int H, int k) {
+  if (total_q < 0 || !mla_heads_ok(H) || k < 1 || k > 4096) return 0;
+  return dsa::indexer_kl_workspace_bytes(total_q, H, k);
+}
+
+dsa_status_t dsa_indexer_kl(const void* q, const void* kv, const int32_t* idx, const float* lse,
+                            const float* logits, int64_t ld_logits, const int32_t* cu_seqlens_q,
+                            const int32_t* cu_seqlens_k, int B, int max_len_q, int max_len_k,
+                            int64_t total_q, int64_t total_k, int H, int d_qk, int k,
+                            float sm_scale, float* kl_out, float* grad_out, float* target_out,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  dsa_status_t st = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_len_q, max_len_k, total_q,
+                                 total_k);
+  if (st != DSA_OK) return st;
+  if (!q || !kv || !idx || !lse || !logits || !kl_out) return DSA_ERR_INVALID_ARG;
+  if (d_qk != 576 || !mla_heads_ok(H) || k < 1 || k > 4096) return DSA_ERR_UNSUPPORTED;
+  if (!(sm_scale > 0.f) || sm_scale != sm_scale) return DSA_ERR_INVALID_ARG;
+  if (ld_logits < max_len_k || ld_logits < 1) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(workspace)) return DSA_ERR_ALIGNMENT;
+  const int64_t groups = (H + 127) / 128;
+  if (total_q * H >= (int64_t(1) << 31) || groups * 4 * total_q * k >= (int64_t(1) << 40) ||
+      total_k >= (int64_t(1) << 31))
+    return DSA_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < dsa_indexer_kl_workspace_size(total_q, H, k))
+    return DSA_ERR_WORKSPACE;
+  if (total_q == 0 || B == 0) return DSA_OK;
+  if (total_k == 0) return DSA_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != DSA_OK) return st;
+  dsa::KlArgs a;
+  a.q = q;
+  a.kv = kv;
+  a.idx = idx;
+  a.lse = lse;
+  a.logits = logits;
+  a.ld = ld_logits;
+  a.cu_q = cu_seqlens_q;
+  a.cu_k = cu_seqlens_k;
+  a.B = B;
+  a.total_q = total_q;
+  a.H = H;
+  a.k = k;
+  a.sm_scale = sm_scale;
+  a.kl = kl_out;
+  a.grad = grad_out;
+  a.target = target_out;
+  a.part = static_cast<float*>(workspace);
+  a.num_sms = dev->num_sms;
+  return from_cuda(
+      dsa::launch_indexer_kl(a, next_err(dev), static_cast<cudaStream_t>(stream)));
+}
+
 size_t dsa_forward_workspace_size(int64_t total_q, int max_len_k, int k) {
   if (total_q < 0 || max_len_k < 0 || k < 1) return 0;
   const int64_t ld = (static_cast<int64_t>(max_len_k) + 3) / 4 * 4;

@@ -48,11 +48,33 @@ struct MlaArgs {
   int num_sms;   // persistent grid size
 };
 
+struct KlArgs {
+  const void* q;
+  const void* kv;
+  const int32_t* idx;
+  const float* lse;
+  const float* logits;
+  int64_t ld;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int B;
+  int64_t total_q;
+  int H, k;
+  float sm_scale;
+  float* kl;
+  float* grad;     // nullable
+  float* target;   // nullable
+  float* part;     // workspace: per-(head group, sub-partition) partial sums
+  int num_sms;
+};
+
 // Each returns cudaSuccess or the launch error.
 cudaError_t launch_indexer(const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
                            const IndexerArgs& a, int num_sms, DevErr err, cudaStream_t s);
 cudaError_t launch_topk(const TopkArgs& a, DevErr err, cudaStream_t s);
 cudaError_t launch_sparse_mla(const void* q, const void* kv, const MlaArgs& a, DevErr err,
                               cudaStream_t s);
+cudaError_t launch_indexer_kl(const KlArgs& a, DevErr err, cudaStream_t s);
+size_t indexer_kl_workspace_bytes(int64_t total_q, int H, int k);
 
 }  // namespace dsa

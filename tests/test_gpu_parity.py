@@ -226,6 +226,87 @@ def test_forward_end_to_end_small_varlen():
         C.check_attention(g_out[q0:q1], o, g_lse[q0:q1], ol)
 
 
+# --------------------------------------------------------------------------
+# The indexer's KL training signal (oracle fed the GPU's scores and indices;
+# the kernel uses the attention's lse, whose parity bar is 1e-3, so the
+# per-head probabilities may differ by that much relatively: 2e-3)
+# --------------------------------------------------------------------------
+
+KL_RTOL = 2e-3
+
+
+def _gpu_kl(gpu, logits, idx, lse):
+    T_q, k = idx.shape
+    kl = torch.full((T_q,), float("nan"), device="cuda")
+    grad = torch.full((T_q, k), float("nan"), device="cuda")
+    tgt = torch.full((T_q, k), float("nan"), device="cuda")
+    dsa.dsa_indexer_kl(gpu.q, gpu.kv, idx, lse, logits, gpu.cu_q, gpu.cu_k, gpu.B, gpu.max_len_q,
+                       gpu.max_len_k, gpu.k, gpu.scale, kl, grad, tgt)
+    C.assert_no_device_error()
+    return C.np_(kl), C.np_(grad), C.np_(tgt)
+
+
+def _kl_vs_oracle(cpu, logits, idx, kl, grad, tgt, rows_of=None):
+    lg = C.np_(logits)
+    gi = C.np_(idx)
+    for b in range(cpu.B):
+        q0, q1, k0, k1 = C.seq_slices(cpu, b)
+        rows = np.arange(q1 - q0) if rows_of is None else rows_of(b)
+        if len(rows) == 0:
+            continue
+        pos = np.array(_p_rows(cpu, b, rows), dtype=np.int64)
+        r_abs = q0 + rows
+        o_kl, o_grad, o_tgt = oracle.indexer_kl_at(
+            C.bits(cpu.q[torch.as_tensor(r_abs)]), C.bits(cpu.kv[k0:k1]), gi[r_abs], pos,
+            lg[r_abs], cpu.scale)
+        scale = np.abs(o_tgt).max(axis=1, keepdims=True) + 1e-12
+        assert np.all(np.abs(tgt[r_abs] - o_tgt) <= KL_RTOL * scale), f"target, sequence {b}"
+        qprob = o_grad + o_tgt
+        gscale = (np.abs(qprob) + np.abs(o_tgt)).max(axis=1, keepdims=True) + 1e-12
+        assert np.all(np.abs(grad[r_abs] - o_grad) <= KL_RTOL * gscale), f"grad, sequence {b}"
+        assert np.all(np.abs(kl[r_abs] - o_kl) <= KL_RTOL * np.abs(o_kl) + 1e-5), f"kl, sequence {b}"
+        invalid = ~((gi[r_abs] >= 0) & (gi[r_abs] <= pos[:, None]))
+        assert np.all(grad[r_abs][invalid] == 0) and np.all(tgt[r_abs][invalid] == 0)
+
+
+@pytest.mark.parametrize("H,k", [(128, 100), (16, 64), (192, 256), (64, 130)])
+def test_indexer_kl_small(H, k):
+    cpu, gpu = _small(H_I=8, d_I=64, H=H, lens=[400, 300], lens_q=[400, 90], k=k, seed=121,
+                      q_div=3.0)
+    logits = C.gpu_indexer(gpu, fill=0.0)
+    idx, _ = C.gpu_topk(gpu, logits, with_val=False)
+    if k >= 100:
+        idx[5:, 3] = -1                  # holes inside the valid prefix
+    _, lse = C.gpu_attention(gpu, idx)
+    kl, grad, tgt = _gpu_kl(gpu, logits, idx, lse)
+    _kl_vs_oracle(cpu, logits, idx, kl, grad, tgt)
+
+
+def test_indexer_kl_dense_warmup_all_keys():
+    # k >= every p + 1: the selection is every causal key (the dense warm-up)
+    cpu, gpu = _small(H_I=8, d_I=64, H=128, L=300, k=320, seed=122, q_div=3.0)
+    logits = C.gpu_indexer(gpu, fill=0.0)
+    idx, _ = C.gpu_topk(gpu, logits, with_val=False)
+    _, lse = C.gpu_attention(gpu, idx)
+    kl, grad, tgt = _gpu_kl(gpu, logits, idx, lse)
+    _kl_vs_oracle(cpu, logits, idx, kl, grad, tgt)
+
+
+def test_indexer_kl_config1_sampled():
+    cpu = W.make_prefill(1)
+    gpu = cpu.to("cuda")
+    logits = C.gpu_indexer(gpu, fill=0.0)
+    idx, _ = C.gpu_topk(gpu, logits, with_val=False)
+    _, lse = C.gpu_attention(gpu, idx)
+    kl, grad, tgt = _gpu_kl(gpu, logits, idx, lse)
+    L, k = cpu.T_q, cpu.k
+    rows = np.array([0, 1, k - 2, k - 1, k, k + 1, 4000, L - 1])
+    lg = torch.zeros(logits.shape, dtype=torch.float32)
+    lg[torch.as_tensor(rows)] = logits[torch.as_tensor(rows, device="cuda")].cpu()
+    del logits
+    _kl_vs_oracle(cpu, lg, idx, kl, grad, tgt, rows_of=lambda b: rows)
+
+
 # Host-buffer entry point: the batch goes through in chunks of query rows on
 # several streams; each row's arithmetic is unchanged, so the results are
 # bitwise those of dsa_forward.  The chunk sizes cut sequences in the middle
