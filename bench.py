@@ -39,6 +39,7 @@ KERNEL_FILES = {
     "indexer_kernel": "sparse_attention_08_b200/csrc/indexer.cu",
     "topk_kernel": "sparse_attention_08_b200/csrc/topk.cu",
     "sparse_mla_kernel": "sparse_attention_08_b200/csrc/sparse_mla.cu",
+    "attn_target_kernel": "sparse_attention_08_b200/csrc/indexer_kl.cu",
 }
 
 
@@ -357,7 +358,8 @@ def run_ours(args):
         kl_extra = {"ms": round(kl_ms, 4), "bound": "tensor",
                     "achieved": round(s_flops / (kl_ms / 1e3) / 1e12, 2), "peak": bf16_peak,
                     "unit": "TFLOP/s", "frac": round(s_flops / (kl_ms / 1e3) / 1e12 / bf16_peak, 4),
-                    "work": "S = Q K^T of every head and selected entry (2*576 flops each)"}
+                    "work": "S = Q K^T of every head and selected entry (2*576 flops each)",
+                    "traffic": ncu_traffic("attn_target_kernel", f"{cfg.name}")}
         del ws_kl, grad
 
     # ---- end to end through dsa_forward with host buffers
