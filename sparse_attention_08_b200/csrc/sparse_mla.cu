@@ -314,8 +314,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           cp_async_commit();
-#pragma unroll
-          for (int pass = 0; pass < 4; ++pass) rows[pass] = load_idx(0, rsub + 16 * pass);
         } else {
 #pragma unroll
           for (int pass = 0; pass < 4; ++pass) {
@@ -326,14 +324,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < kChunks; ++c) cp_async16(dst + c * kChunkBytes, src + c * 64);
           }
           cp_async_commit();
-          if (j + 1 < it.nb) {                                       // next block's rows
-#pragma unroll
-            for (int pass = 0; pass < 4; ++pass) rows[pass] = load_idx(j + 1, rsub + 16 * pass);
-          }
         }
         cp_async_wait_all();
         fence_proxy_async_smem();
         mbar_arrive(kv_full(st));
+        // the next block's rows, loaded after the arrive: its release
+        // semantics would otherwise hold the slot back until they land
+        if (j + 1 < it.nb) {
+#pragma unroll
+          for (int pass = 0; pass < 4; ++pass) rows[pass] = load_idx(j + 1, rsub + 16 * pass);
+        }
       }
     }
   } else if (warp == kMmaWarp || warp == kPvWarp) {
@@ -446,15 +446,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < it.nb; ++j, ++u, ++gb) {
         const uint32_t sb = gb & 1;            // S buffer
         const uint32_t st = u % kStages;       // slot (P goes over its RoPE chunk)
-        const uint32_t vmask_lo = __ballot_sync(0xffffffffu, nx0);
-        const uint32_t vmask_hi = __ballot_sync(0xffffffffu, nx1);
-        if (j + 1 < it.nb) {
-          nx0 = entry_ok(it, (j + 1) * kBlockN + 2 * lane);
-          nx1 = entry_ok(it, (j + 1) * kBlockN + 2 * lane + 1);
-        } else if (wn < P.n_items) {
-          nx0 = entry_ok(nit, 2 * lane);
-          nx1 = entry_ok(nit, 2 * lane + 1);
-        }
         if (!warp_wait(s_full(sb), (gb >> 1) & 1, P.err)) {
           ok = false;
           break;
@@ -466,6 +457,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free(sb));
+        const uint32_t vmask_lo = __ballot_sync(0xffffffffu, nx0);
+        const uint32_t vmask_hi = __ballot_sync(0xffffffffu, nx1);
 
         // key of register 4i+e (row a) and 4i+2+e (row b): 8i + 2qd + e.
         // Entries outside the selection get the raw score -inf; full blocks
@@ -569,6 +562,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full(st));
+        // validity of the next block's entries, loaded after the arrive (its
+        // release semantics would otherwise wait for them)
+        if (j + 1 < it.nb) {
+          nx0 = entry_ok(it, (j + 1) * kBlockN + 2 * lane);
+          nx1 = entry_ok(it, (j + 1) * kBlockN + 2 * lane + 1);
+        } else if (wn < P.n_items) {
+          nx0 = entry_ok(nit, 2 * lane);
+          nx1 = entry_ok(nit, 2 * lane + 1);
+        }
       }
       if (!ok) break;
       // ---- row statistics for the output warps
