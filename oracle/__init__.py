@@ -15,6 +15,8 @@ indexer works"; "DeepSeek-V3.2" atlas entry, "Design overview"):
 * indexer  I[t,s] = sum_j w[t,j] * ReLU(qhat[t,j] . khat[s])  for s <= p
 * top-k    the min(k, p+1) best scores, ties to the lower index, ascending
 * attention softmax over the selected latents, shared by all query heads
+* masked MHA  dense per-head attention restricted to the selected set (the
+  short-prefill mode the "DeepSeek-V3.2" paper record names)
 """
 from __future__ import annotations
 
@@ -73,6 +75,9 @@ def _load():
         lib.oracle_indexer_kl_at.argtypes = [P, P, P, P, P, i64, i64, i64, i32, i32, i32,
                                              ctypes.c_double, P, P, P]
         lib.oracle_indexer_kl_at.restype = i32
+        lib.oracle_masked_mha_at.restype = i32
+        lib.oracle_masked_mha_at.argtypes = [P, P, P, P, P, i64, i64, i32, i32, i32, i32,
+                                             ctypes.c_double, P, P]
         lib.oracle_num_threads.argtypes = []
         _lib = lib
     return _lib
@@ -276,3 +281,30 @@ def indexer_kl_at(q_bits, kv_bits, idx, pos, logits, scale):
     if rc != 0:
         raise ValueError("oracle_indexer_kl_at: bad arguments")
     return kl, grad, target
+
+
+def masked_mha_at(q_bits, k_bits, v_bits, idx, pos, scale):
+    """The masked MHA mode ("DeepSeek-V3.2" paper record: short-sequence
+    prefilling uses a masked MHA mode that simulates DSA): per-head dense
+    attention of query row r (position pos[r]) over the set of its valid
+    selected keys.  q_bits [R, H, d_qk], k_bits [n_k, H, d_qk], v_bits
+    [n_k, H, d_v] (bf16 bits), idx [R, topk].  Returns (out [R, H, d_v],
+    lse [R, H]) in fp64."""
+    q_bits = _c(q_bits, np.uint16)
+    k_bits = _c(k_bits, np.uint16)
+    v_bits = _c(v_bits, np.uint16)
+    idx = _c(idx, np.int32)
+    pos = _c(pos, np.int64)
+    R, H, d_qk = q_bits.shape
+    n_k = k_bits.shape[0]
+    d_v = v_bits.shape[2]
+    if k_bits.shape != (n_k, H, d_qk) or v_bits.shape[:2] != (n_k, H) or idx.shape[0] != R:
+        raise ValueError("masked_mha_at: shape mismatch")
+    out = np.empty((R, H, d_v), dtype=np.float64)
+    lse = np.empty((R, H), dtype=np.float64)
+    rc = _load().oracle_masked_mha_at(_ptr(q_bits), _ptr(k_bits), _ptr(v_bits), _ptr(idx), _ptr(pos),
+                                      R, n_k, H, d_qk, d_v, int(idx.shape[1]), float(scale),
+                                      _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_masked_mha_at: bad arguments")
+    return out, lse

@@ -80,3 +80,26 @@ def attention_loops(q_row, kv, sel, scale, d_v):
             out[h] += (e / z) * kv[s, :d_v]
         lse[h] = m + math.log(z)
     return out, lse
+
+
+def masked_mha_loops(q_row, k, v, entries, p, scale):
+    """Masked MHA mode by explicit loops: q_row float64 [H, d_qk], k float64
+    [n_k, H, d_qk], v float64 [n_k, H, d_v]; entries is the raw index row.
+    The selected set is built with a Python set (valid entries 0 <= s <= p,
+    repeats once); each head takes a softmax over it with math.exp.  Returns
+    (out [H, d_v], lse [H]); an empty set gives zeros and -inf."""
+    sel = sorted({int(s) for s in entries if 0 <= int(s) <= p})
+    H, d_v = q_row.shape[0], v.shape[2]
+    out = np.zeros((H, d_v))
+    lse = np.full(H, -math.inf)
+    if not sel:
+        return out, lse
+    for h in range(H):
+        xs = [scale * math.fsum(float(a) * float(b) for a, b in zip(q_row[h], k[s, h])) for s in sel]
+        m = max(xs)
+        es = [math.exp(x - m) for x in xs]
+        z = math.fsum(es)
+        for e, s in zip(es, sel):
+            out[h] += (e / z) * v[s, h]
+        lse[h] = m + math.log(z)
+    return out, lse

@@ -503,6 +503,83 @@ int oracle_indexer_kl_at(const uint16_t* q, const uint16_t* kv, const int32_t* i
   return bad ? -1 : 0;
 }
 
+/* ---------------------------------------------------------------------- */
+/* Masked MHA mode.                                                         */
+/* ---------------------------------------------------------------------- */
+
+/* The masked MHA mode that stands in for DSA on short prefills ("DeepSeek-
+ * V3.2" paper record: short-sequence prefilling uses a masked MHA mode that
+ * simulates DSA; the pages name it without detail).  Reading: dense attention
+ * in the MHA form of MLA (every head has its own key and value), restricted
+ * by a mask to the query's selected set S = { idx[r, j] : 0 <= idx[r, j] <= p }
+ * taken as a set (a repeated entry counts once), keys visited in ascending
+ * order:
+ *     out[r,h,:] = sum_{s in S} softmax_s(scale * q[r,h,:] . k[s,h,:]) v[s,h,:]
+ *     lse[r,h]   = log sum_{s in S} exp(scale * q[r,h,:] . k[s,h,:]).
+ * q: n_rows x H x d_qk (row r at position pos[r]); k: n_k x H x d_qk;
+ * v: n_k x H x d_v, all bf16 bits; idx: n_rows x topk.  A row with empty S
+ * gets out = 0, lse = -inf. */
+int oracle_masked_mha_at(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                         const int32_t* idx, const int64_t* pos, int64_t n_rows, int64_t n_k,
+                         int H, int d_qk, int d_v, int topk, double scale, double* out,
+                         double* lse) {
+  if (topk <= 0 || H <= 0 || d_qk <= 0 || d_v <= 0 || !pos || n_k <= 0) return -1;
+  int bad = 0;
+#pragma omp parallel
+  {
+    unsigned char* mark = (unsigned char*)calloc((size_t)n_k, 1);
+    double* x = (double*)malloc(sizeof(double) * (size_t)n_k);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; ++r) {
+      const int64_t p = pos[r];
+      if (p < 0 || p >= n_k || !mark || !x) {
+        bad = 1;
+        continue;
+      }
+      const int32_t* row = idx + r * (int64_t)topk;
+      int64_t n_sel = 0;
+      for (int j = 0; j < topk; ++j)
+        if (row[j] >= 0 && row[j] <= p && !mark[row[j]]) {
+          mark[row[j]] = 1;
+          ++n_sel;
+        }
+      for (int h = 0; h < H; ++h) {
+        const uint16_t* qh = q + (r * H + h) * (int64_t)d_qk;
+        double* oh = out + (r * H + h) * (int64_t)d_v;
+        for (int d = 0; d < d_v; ++d) oh[d] = 0.0;
+        if (n_sel == 0) {
+          lse[r * H + h] = -INFINITY;
+          continue;
+        }
+        double m = -INFINITY;
+        for (int64_t s = 0; s <= p; ++s) {
+          if (!mark[s]) continue;
+          const uint16_t* ks = k + (s * H + h) * (int64_t)d_qk;
+          double dot = 0.0;
+          for (int d = 0; d < d_qk; ++d) dot += oracle_bf16_decode(qh[d]) * oracle_bf16_decode(ks[d]);
+          x[s] = scale * dot;
+          if (x[s] > m) m = x[s];
+        }
+        double z = 0.0;
+        for (int64_t s = 0; s <= p; ++s) {
+          if (!mark[s]) continue;
+          const double e = exp(x[s] - m);
+          z += e;
+          const uint16_t* vs = v + (s * H + h) * (int64_t)d_v;
+          for (int d = 0; d < d_v; ++d) oh[d] += e * oracle_bf16_decode(vs[d]);
+        }
+        for (int d = 0; d < d_v; ++d) oh[d] /= z;
+        lse[r * H + h] = m + log(z);
+      }
+      for (int j = 0; j < topk; ++j)
+        if (row[j] >= 0 && row[j] <= p) mark[row[j]] = 0;
+    }
+    free(mark);
+    free(x);
+  }
+  return bad ? -1 : 0;
+}
+
 /* Threads OpenMP will use (reported beside the CPU baseline). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

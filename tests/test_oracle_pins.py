@@ -444,3 +444,112 @@ def test_kl_target_is_the_mean_of_the_single_head_targets_and_matches_attention(
         mix = sum(heads[0][r, j] * vals[idx[r, j]] for j in range(idx.shape[1])
                   if heads[0][r, j] > 0)
         assert np.allclose(mix, out[r, 0], atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Masked MHA mode ("DeepSeek-V3.2" paper record: short-sequence prefilling
+# uses a masked MHA mode that simulates DSA).  Reading: dense per-head
+# attention restricted to the selected set.
+
+def _mha_case(n=40, H=3, d_qk=24, d_v=8, seed=5):
+    g = torch.Generator().manual_seed(seed)
+    q = (torch.randn(n, H, d_qk, generator=g) / 3).to(torch.bfloat16)
+    k = torch.randn(n, H, d_qk, generator=g).to(torch.bfloat16)
+    v = torch.randn(n, H, d_v, generator=g).to(torch.bfloat16)
+    return q, k, v
+
+
+def test_masked_mha_all_causal_keys_selected_is_causal_sdpa():
+    """Every earlier key selected (p + 1 <= topk): the masked mode is plain
+    causal multi-head attention, which torch computes in fp64."""
+    n, H, scale = 40, 3, 0.3
+    q, k, v = _mha_case(n, H)
+    topk = 48
+    rng = np.random.default_rng(1)
+    idx = np.full((n, topk), -1, dtype=np.int32)
+    for t in range(n):
+        sel = rng.permutation(t + 1)
+        idx[t, :t + 1] = sel
+    out, lse = oracle.masked_mha_at(_bits(q), _bits(k), _bits(v), idx, np.arange(n), scale)
+    qd, kd, vd = (x.to(torch.float64).transpose(0, 1) for x in (q, k, v))   # [H, n, d]
+    ref = torch.nn.functional.scaled_dot_product_attention(qd, kd, vd, is_causal=True, scale=scale)
+    np.testing.assert_allclose(out, ref.transpose(0, 1).numpy(), rtol=1e-12, atol=1e-12)
+    sc = scale * qd @ kd.transpose(1, 2)
+    sc = sc.masked_fill(torch.ones(n, n, dtype=torch.bool).triu(1), -math.inf)
+    np.testing.assert_allclose(lse, torch.logsumexp(sc, dim=-1).transpose(0, 1).numpy(), rtol=1e-12,
+                               atol=1e-12)
+
+
+def test_masked_mha_matches_explicit_loops_with_repeats_and_invalid_entries():
+    n, H = 30, 2
+    q, k, v = _mha_case(n, H, d_qk=16, d_v=8, seed=9)
+    rng = np.random.default_rng(3)
+    topk = 12
+    idx = rng.integers(-3, n + 3, size=(n, topk)).astype(np.int32)
+    idx[:, 5] = idx[:, 4]                                   # a repeated entry counts once
+    idx[7, :] = -1                                          # an empty selection
+    pos = np.arange(n)
+    out, lse = oracle.masked_mha_at(_bits(q), _bits(k), _bits(v), idx, pos, 0.25)
+    qf, kf, vf = (x.to(torch.float64).numpy() for x in (q, k, v))
+    for t in range(n):
+        o_ref, l_ref = brute.masked_mha_loops(qf[t], kf, vf, idx[t], t, 0.25)
+        np.testing.assert_allclose(out[t], o_ref, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(lse[t], l_ref, rtol=1e-12)
+    assert np.all(out[7] == 0) and np.all(np.isneginf(lse[7]))
+
+
+def test_masked_mha_ignores_keys_outside_the_selection():
+    """A key that is not selected may carry any score: the result does not move."""
+    n, H = 24, 2
+    q, k, v = _mha_case(n, H, d_qk=16, d_v=8, seed=4)
+    idx = np.array([[s for s in range(0, t + 1, 2)] + [-1] * (12 - len(range(0, t + 1, 2)))
+                    for t in range(n)], dtype=np.int32)
+    a = oracle.masked_mha_at(_bits(q), _bits(k), _bits(v), idx, np.arange(n), 0.5)
+    k2 = k.clone()
+    k2[1::2] = (q[1::2] * 40).to(torch.bfloat16)           # odd keys: huge, unselected
+    b = oracle.masked_mha_at(_bits(q), _bits(k2), _bits(v), idx, np.arange(n), 0.5)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_masked_mha_is_the_mqa_mode_after_absorption():
+    """The MHA and MQA forms of MLA give the same attention: with per-head keys
+    k_h = [W_UK_h^T c_nope ; c_rope], values v_h = W_UV_h^T c_nope and the
+    absorbed query q_abs = [W_UK_h q_nope ; q_rope], the MHA output of head h
+    is W_UV_h^T applied to the MQA output over the latents.  The projections
+    are signed selections of latent dims, so every product is exact in bf16
+    and the identity holds to fp64 rounding."""
+    rng = np.random.default_rng(7)
+    n_k, H, dn, dr, dl = 50, 3, 16, 8, 64           # nope, rope, latent dims (latent > heads' dims)
+    R, topk, scale = 6, 20, 0.2
+    g = torch.Generator().manual_seed(2)
+    c = torch.randn(n_k, dl + dr, generator=g).to(torch.bfloat16)            # [c_nope ; c_rope]
+    q_nope = (torch.randn(R, H, dn, generator=g) / 2).to(torch.bfloat16)
+    q_rope = (torch.randn(R, H, dr, generator=g) / 2).to(torch.bfloat16)
+    k_h = torch.zeros(n_k, H, dn + dr, dtype=torch.bfloat16)
+    v_h = torch.zeros(n_k, H, dn, dtype=torch.bfloat16)
+    q_abs = torch.zeros(R, H, dl + dr, dtype=torch.bfloat16)
+    w_uv = np.zeros((H, dn, dl))                     # W_UV_h^T as a matrix: v_h = w_uv[h] @ c_nope
+    for h in range(H):
+        uk = rng.permutation(dl)[:dn]
+        sk = rng.choice([-1.0, 1.0], size=dn)
+        uv = rng.permutation(dl)[:dn]
+        sv = rng.choice([-1.0, 1.0], size=dn)
+        for j in range(dn):
+            k_h[:, h, j] = c[:, uk[j]] * sk[j]
+            q_abs[:, h, uk[j]] = q_nope[:, h, j] * sk[j]
+            v_h[:, h, j] = c[:, uv[j]] * sv[j]
+            w_uv[h, j, uv[j]] = sv[j]
+        k_h[:, h, dn:] = c[:, dl:]
+        q_abs[:, h, dl:] = q_rope[:, h]
+    q_mha = torch.cat([q_nope, q_rope], dim=2)
+    pos = np.array([49, 30, 12, 40, 5, 25])
+    idx = np.full((R, topk), -1, dtype=np.int32)
+    for r, p in enumerate(pos):
+        sel = np.sort(rng.permutation(p + 1)[:min(topk, p + 1)])
+        idx[r, :len(sel)] = sel
+    out_mha, lse_mha = oracle.masked_mha_at(_bits(q_mha), _bits(k_h), _bits(v_h), idx, pos, scale)
+    out_mqa, lse_mqa = oracle.sparse_mla_at(_bits(q_abs), _bits(c), idx, pos, scale, d_v=dl)
+    np.testing.assert_allclose(lse_mha, lse_mqa, rtol=1e-12, atol=1e-12)
+    for h in range(H):
+        np.testing.assert_allclose(out_mha[:, h], out_mqa[:, h] @ w_uv[h].T, rtol=1e-11, atol=1e-12)
