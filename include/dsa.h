@@ -270,6 +270,43 @@ DSA_API dsa_status_t dsa_indexer_kl(const void* q, const void* kv, const int32_t
  * [total_q, k] f32 per group of 128 heads.  Returns 0 for invalid sizes. */
 DSA_API size_t dsa_indexer_kl_workspace_size(int64_t total_q, int H, int k);
 
+/*
+ * The masked MHA mode ("DeepSeek-V3.2" paper record: short-sequence
+ * prefilling uses a masked MHA mode that simulates DSA; the pages give no
+ * detail, so it is read as dense attention in the MHA form of MLA -- per-head
+ * keys and values -- restricted by a mask to each query's selected set):
+ *
+ *   out[q_row, h, :] = sum_{s in S} softmax_s(sm_scale * q[q_row,h,:] . k[k_row(s),h,:])
+ *                                   * v[k_row(s), h, :]
+ *   lse[q_row, h]    = log sum_{s in S} exp(sm_scale * q[q_row,h,:] . k[k_row(s),h,:])
+ *
+ * S is the SET of entries among the first min(topk, p+1) of idx[q_row, :]
+ * with 0 <= s <= p (a repeated entry counts once); keys are visited densely,
+ * so the cost is that of causal attention, whatever S holds.  A row with an
+ * empty S gets out = 0 and lse = -inf.
+ *
+ *  q        (device) bf16 [total_q, H, 192]: 128 dims + 64 RoPE dims per head
+ *  k        (device) bf16 [total_k, H, 192]
+ *  v        (device) bf16 [total_k, H, 128]
+ *  idx      (device) int32 [total_q, topk] (dsa_topk's output fits)
+ *  out      (device) bf16 [total_q, H, 128]
+ *  lse      (device, nullable) f32 [total_q, H] (natural log)
+ *  workspace (device) dsa_masked_mha_workspace_size bytes: the selection as a
+ *           bitmask, rebuilt by every call
+ *  Supported: d_qk = 192, d_v = 128, 1 <= H <= 65535, max_len_k <= 131072.
+ *  Arithmetic: bf16 tensor-core products, fp32 accumulation and softmax.
+ */
+DSA_API dsa_status_t dsa_masked_mha_fwd(const void* q, const void* k, const void* v,
+                                        const int32_t* idx, const int32_t* cu_seqlens_q,
+                                        const int32_t* cu_seqlens_k, int B, int max_len_q,
+                                        int max_len_k, int64_t total_q, int64_t total_k, int H,
+                                        int d_qk, int d_v, int topk, float sm_scale, void* out,
+                                        float* lse, void* workspace, size_t workspace_bytes,
+                                        void* stream);
+
+/* Device workspace bytes for dsa_masked_mha_fwd (0 for invalid sizes). */
+DSA_API size_t dsa_masked_mha_workspace_size(int64_t total_q, int max_len_k);
+
 /* Bytes of workspace dsa_forward needs: an f32 score matrix [total_q,
  * round_up(max_len_k, 4)] plus an int32 index matrix [total_q, k], each
  * 256-byte aligned.  Returns 0 for invalid sizes. */

@@ -16,7 +16,8 @@ __all__ = [
     "dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward",
     "dsa_forward_workspace_size", "dsa_get_device_error", "dsa_forward_noalloc",
     "dsa_forward_host", "dsa_forward_host_workspace_size", "dsa_indexer_kl",
-    "dsa_indexer_kl_workspace_size", "EXPORTED",
+    "dsa_indexer_kl_workspace_size", "dsa_masked_mha_fwd", "dsa_masked_mha_workspace_size",
+    "EXPORTED",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -28,7 +29,8 @@ EXPORTED = (
     "dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward",
     "dsa_forward_workspace_size", "dsa_status_string", "dsa_get_device_error", "dsa_version",
     "dsa_forward_noalloc", "dsa_forward_host", "dsa_forward_host_workspace_size",
-    "dsa_indexer_kl", "dsa_indexer_kl_workspace_size",
+    "dsa_indexer_kl", "dsa_indexer_kl_workspace_size", "dsa_masked_mha_fwd",
+    "dsa_masked_mha_workspace_size",
 )
 
 STATUS = {
@@ -72,6 +74,11 @@ def load():
     lib.dsa_indexer_kl.restype = I
     lib.dsa_indexer_kl_workspace_size.argtypes = [I64, I, I]
     lib.dsa_indexer_kl_workspace_size.restype = ctypes.c_size_t
+    lib.dsa_masked_mha_fwd.argtypes = [P, P, P, P, P, P, I, I, I, I64, I64, I, I, I, I, F, P, P, P,
+                                       ctypes.c_size_t, P]
+    lib.dsa_masked_mha_fwd.restype = I
+    lib.dsa_masked_mha_workspace_size.argtypes = [I64, I]
+    lib.dsa_masked_mha_workspace_size.restype = ctypes.c_size_t
     lib.dsa_forward_host_workspace_size.argtypes = [I64, I, I, I, I, I, I, I, I]
     lib.dsa_forward_host_workspace_size.restype = ctypes.c_size_t
     for name in ("dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward",
@@ -326,6 +333,36 @@ def dsa_indexer_kl(q, kv, idx, lse, logits, cu_seqlens_q, cu_seqlens_k, B, max_l
                                _ptr(target_out), _ptr(workspace), int(workspace.numel()),
                                _stream(stream))
     _check(rc, "dsa_indexer_kl")
+
+
+def dsa_masked_mha_workspace_size(total_q, max_len_k) -> int:
+    return int(load().dsa_masked_mha_workspace_size(int(total_q), int(max_len_k)))
+
+
+def dsa_masked_mha_fwd(q, k, v, idx, cu_seqlens_q, cu_seqlens_k, B, max_len_q, max_len_k,
+                       topk, sm_scale, out, lse=None, workspace=None, stream=None):
+    """The masked MHA mode (see include/dsa.h): dense per-head attention of
+    q [T_q, H, 192] over k [T_k, H, 192], v [T_k, H, 128], restricted to each
+    query's selected set idx [T_q, topk]; writes out [T_q, H, 128] (bf16) and
+    lse [T_q, H] (fp32, optional).  `workspace` (uint8 CUDA tensor) is
+    allocated here when not given."""
+    import torch
+    _need(q, torch.bfloat16, "q", 3)
+    _need(k, torch.bfloat16, "k", 3)
+    _need(v, torch.bfloat16, "v", 3)
+    _need(idx, torch.int32, "idx", 2)
+    _need(out, torch.bfloat16, "out", 3)
+    _need(lse, torch.float32, "lse", 2)
+    T_q, H, d_qk = q.shape
+    nbytes = dsa_masked_mha_workspace_size(T_q, max_len_k)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    rc = load().dsa_masked_mha_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(cu_seqlens_q),
+                                   _ptr(cu_seqlens_k), int(B), int(max_len_q), int(max_len_k),
+                                   int(T_q), int(k.shape[0]), int(H), int(d_qk), int(v.shape[2]),
+                                   int(topk), float(sm_scale), _ptr(out), _ptr(lse),
+                                   _ptr(workspace), int(workspace.numel()), _stream(stream))
+    _check(rc, "dsa_masked_mha_fwd")
 
 
 def dsa_get_device_error(stream=None) -> int:

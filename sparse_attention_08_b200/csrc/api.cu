@@ -81,6 +81,21 @@ dsa_status_t encode_2d(CUtensorMap* m, CUtensorMapDataType dtype, const void* ba
   return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_CUDA;
 }
 
+// Row-major 3D tensor [d2, d1, d0] (d0 innermost) of bf16, box of
+// box0 x 1 x box2 elements, 128-byte swizzle.
+dsa_status_t encode_3d_bf16(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                            uint32_t box0, uint32_t box2) {
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  const cuuint32_t box[3] = {box0, 1, box2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_CUDA;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 dsa_status_t check_varlen(const int32_t* cu_q, const int32_t* cu_k, int B, int max_len_q,
@@ -242,6 +257,60 @@ dsa_status_t dsa_sparse_mla_fwd(const void* q, const void* kv, const int32_t* id
   a.num_sms = dev->num_sms;
   return from_cuda(
       dsa::launch_sparse_mla(q, kv, a, next_err(dev), static_cast<cudaStream_t>(stream)));
+}
+
+size_t dsa_masked_mha_workspace_size(int64_t total_q, int max_len_k) {
+  if (total_q < 0 || max_len_k < 1 || max_len_k > 131072) return 0;
+  return dsa::masked_mha_workspace_bytes(total_q, max_len_k);
+}
+
+dsa_status_t dsa_masked_mha_fwd(const void* q, const void* k, const void* v, const int32_t* idx,
+                                const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
+                                int max_len_q, int max_len_k, int64_t total_q, int64_t total_k,
+                                int H, int d_qk, int d_v, int topk, float sm_scale, void* out,
+                                float* lse, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  dsa_status_t st = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_len_q, max_len_k, total_q,
+                                 total_k);
+  if (st != DSA_OK) return st;
+  if (!q || !k || !v || !idx || !out) return DSA_ERR_INVALID_ARG;
+  if (d_qk != 192 || d_v != 128 || H < 1 || H > 65535 || topk < 1 || topk > 131072 ||
+      max_len_k > 131072)
+    return DSA_ERR_UNSUPPORTED;
+  if (!(sm_scale > 0.f) || sm_scale != sm_scale) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(out) ||
+      (lse && !aligned16(lse)) || (workspace && !aligned16(workspace)))
+    return DSA_ERR_ALIGNMENT;
+  if (total_q * H >= (int64_t(1) << 31) || total_k >= (int64_t(1) << 31) ||
+      (int64_t)B * ((max_len_q + 127) / 128) >= (int64_t(1) << 31))
+    return DSA_ERR_UNSUPPORTED;
+  if (total_q == 0 || B == 0) return DSA_OK;
+  if (total_k == 0) return DSA_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < dsa::masked_mha_workspace_bytes(total_q, max_len_k))
+    return DSA_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != DSA_OK) return st;
+  CUtensorMap tq, tk, tv;
+  if ((st = encode_3d_bf16(&tq, q, 192, H, total_q, 64, 128)) != DSA_OK) return st;
+  if ((st = encode_3d_bf16(&tk, k, 192, H, total_k, 64, 128)) != DSA_OK) return st;
+  if ((st = encode_3d_bf16(&tv, v, 128, H, total_k, 64, 128)) != DSA_OK) return st;
+  dsa::MaskedMhaArgs a;
+  a.idx = idx;
+  a.cu_q = cu_seqlens_q;
+  a.cu_k = cu_seqlens_k;
+  a.B = B;
+  a.max_len_q = max_len_q;
+  a.max_len_k = max_len_k;
+  a.total_q = total_q;
+  a.total_k = total_k;
+  a.H = H;
+  a.k = topk;
+  a.sm_scale = sm_scale;
+  a.mask = static_cast<uint32_t*>(workspace);
+  a.out = out;
+  a.lse = lse;
+  return from_cuda(dsa::launch_masked_mha(tq, tk, tv, a, next_err(dev),
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 size_t dsa_indexer_kl_workspace_size(int64_t total_q, int H, int k) {

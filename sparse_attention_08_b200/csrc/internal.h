@@ -75,6 +75,23 @@ cudaError_t launch_topk(const TopkArgs& a, DevErr err, cudaStream_t s);
 cudaError_t launch_sparse_mla(const void* q, const void* kv, const MlaArgs& a, DevErr err,
                               cudaStream_t s);
 cudaError_t launch_indexer_kl(const KlArgs& a, DevErr err, cudaStream_t s);
+
+struct MaskedMhaArgs {
+  const int32_t* idx;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int B, max_len_q, max_len_k;
+  int64_t total_q, total_k;
+  int H, k;
+  float sm_scale;
+  uint32_t* mask;   // workspace: [total_q, masked_mha_workspace_bytes / total_q / 4] words
+  void* out;
+  float* lse;
+};
+
+cudaError_t launch_masked_mha(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                              const MaskedMhaArgs& a, DevErr err, cudaStream_t s);
+size_t masked_mha_workspace_bytes(int64_t total_q, int max_len_k);
 size_t indexer_kl_workspace_bytes(int64_t total_q, int H, int k);
 
 }  // namespace dsa

@@ -341,3 +341,86 @@ def make_small(H_I=4, d_I=64, H=16, L=300, k=64, seed=7, integer=False, device="
                     cu_q=torch.tensor(cu_q, dtype=torch.int32, device=device),
                     cu_k=torch.tensor(cu_k, dtype=torch.int32, device=device),
                     lens_q=lens_qq, lens_k=lens_k, k=k)
+
+
+# ---------------------------------------------------------------------------
+# Masked MHA mode ("DeepSeek-V3.2" paper record: short-sequence prefilling
+# uses a masked MHA mode that simulates DSA).  Per-head queries and keys of
+# 192 dims (128 + 64 RoPE) and values of 128 dims, the MHA form of MLA.
+
+D_QK_MHA = 192
+D_V_MHA = 128
+
+
+@dataclass
+class MhaInputs:
+    q: torch.Tensor        # bf16 [T_q, H, 192]
+    k: torch.Tensor        # bf16 [T_k, H, 192]
+    v: torch.Tensor        # bf16 [T_k, H, 128]
+    idx: torch.Tensor      # int32 [T_q, topk]: a drawn selection, ascending, -1 padded
+    cu_q: torch.Tensor
+    cu_k: torch.Tensor
+    lens_q: list
+    lens_k: list
+    topk: int
+    scale: float
+
+    @property
+    def B(self):
+        return len(self.lens_k)
+
+    @property
+    def T_q(self):
+        return int(sum(self.lens_q))
+
+    @property
+    def max_len_q(self):
+        return max(self.lens_q)
+
+    @property
+    def max_len_k(self):
+        return max(self.lens_k)
+
+
+def make_mha(lens, lens_q=None, H=128, topk=2048, seed=BASE_SEED + 900, device="cpu",
+             q_div=None) -> MhaInputs:
+    """Inputs of the masked MHA mode: q ~ N(0,1)/q_div (default sqrt(192)),
+    k, v ~ N(0,1), all bf16, and a selection per query row at position p:
+    min(topk, p+1) distinct keys of [0, p] drawn uniformly at random (every
+    key when p+1 <= topk), ascending, padded with -1.  Queries of a sequence
+    are its last len_q positions.  Softmax scale 1/sqrt(192).  Draw order:
+    q, k, v, selection noise."""
+    g = _gen(device, seed)
+    lens_k = list(lens)
+    lens_qq = list(lens_k) if lens_q is None else list(lens_q)
+    T_q, T_k = sum(lens_qq), sum(lens_k)
+    q = _bf16_normal((T_q, H, D_QK_MHA), g, device,
+                     div=math.sqrt(D_QK_MHA) if q_div is None else q_div, rows_per_draw=256)
+    k = _bf16_normal((T_k, H, D_QK_MHA), g, device, rows_per_draw=256)
+    v = _bf16_normal((T_k, H, D_V_MHA), g, device, rows_per_draw=256)
+    idx = torch.full((T_q, topk), -1, dtype=torch.int32, device=device)
+    q_row = 0
+    for lq, lk in zip(lens_qq, lens_k):
+        pos = torch.arange(lk - lq, lk, device=device)
+        for r0 in range(0, lq, 1024):
+            r1 = min(lq, r0 + 1024)
+            # uniform noise over the keys; keys past a row's position get +inf,
+            # the topk smallest are a uniform random subset of [0, p]
+            noise = torch.rand((r1 - r0, lk), generator=g, device=device)
+            noise.masked_fill_(torch.arange(lk, device=device)[None, :] > pos[r0:r1, None], 2.0)
+            n = min(topk, lk)
+            sel = torch.topk(noise, n, dim=1, largest=False).indices
+            sel = torch.where(torch.gather(noise, 1, sel) < 2.0, sel, torch.full_like(sel, lk))
+            sel = torch.sort(sel, dim=1).values
+            sel = torch.where(sel >= lk, torch.full_like(sel, -1), sel)
+            idx[q_row + r0:q_row + r1, :n] = sel.to(torch.int32)
+        q_row += lq
+    cu_q, cu_k = [0], [0]
+    for a, b in zip(lens_qq, lens_k):
+        cu_q.append(cu_q[-1] + a)
+        cu_k.append(cu_k[-1] + b)
+    return MhaInputs(q=q, k=k, v=v, idx=idx,
+                     cu_q=torch.tensor(cu_q, dtype=torch.int32, device=device),
+                     cu_k=torch.tensor(cu_k, dtype=torch.int32, device=device),
+                     lens_q=lens_qq, lens_k=lens_k, topk=topk,
+                     scale=1.0 / math.sqrt(D_QK_MHA))

@@ -150,3 +150,26 @@ def test_device_error_word_starts_clear():
     import torch
     torch.zeros(1, device="cuda")
     assert dsa.dsa_get_device_error() == OK
+
+
+def test_masked_mha_checks_before_any_device_call():
+    """Argument checks of the masked MHA mode run on the host."""
+    lib = dsa.load()
+    p = _fake()
+    f = ctypes.c_float(1.0 / 192 ** 0.5)
+    need = dsa.dsa_masked_mha_workspace_size(256, 256)
+    assert need == 256 * 8 * 4                       # 8 words of 32 keys per row
+    assert dsa.dsa_masked_mha_workspace_size(256, 0) == 0
+    assert dsa.dsa_masked_mha_workspace_size(256, 131073) == 0
+
+    def call(d_qk=192, d_v=128, H=4, topk=64, ws=p, nbytes=need, scale=f, q=p):
+        return lib.dsa_masked_mha_fwd(q, p, p, p, p, p, 1, 256, 256, 256, 256, H, d_qk, d_v, topk,
+                                      scale, p, None, ws, nbytes, None)
+    assert call(d_qk=576) == UNSUPPORTED
+    assert call(d_v=512) == UNSUPPORTED
+    assert call(topk=0) == UNSUPPORTED
+    assert call(scale=ctypes.c_float(-1.0)) == INVALID
+    assert call(q=None) == INVALID
+    assert call(ws=None) == WORKSPACE
+    assert call(nbytes=need - 1) == WORKSPACE
+    assert call(q=_fake(0x10008)) == ALIGN
