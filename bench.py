@@ -40,6 +40,7 @@ KERNEL_FILES = {
     "topk_kernel": "sparse_attention_08_b200/csrc/topk.cu",
     "sparse_mla_kernel": "sparse_attention_08_b200/csrc/sparse_mla.cu",
     "attn_target_kernel": "sparse_attention_08_b200/csrc/indexer_kl.cu",
+    "masked_mha_kernel": "sparse_attention_08_b200/csrc/masked_mha.cu",
 }
 
 
@@ -58,6 +59,7 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kl", action="store_true")
+    ap.add_argument("--no-mha", action="store_true")
     return ap.parse_args()
 
 
@@ -362,6 +364,42 @@ def run_ours(args):
                     "traffic": ncu_traffic("attn_target_kernel", f"{cfg.name}")}
         del ws_kl, grad
 
+    # ---- the masked MHA short-prefill mode (not part of the step): dense
+    # per-head attention over the selection, on its own short-prefill workload
+    mha_extra = None
+    if not args.no_mha and world == 1:
+        L_m = 4096
+        mh = W.make_mha([L_m], None, H=128, topk=2048, device="cuda")
+        m_out = torch.empty((mh.T_q, 128, W.D_V_MHA), dtype=torch.bfloat16, device="cuda")
+        m_lse = torch.empty((mh.T_q, 128), dtype=torch.float32, device="cuda")
+        m_ws = torch.empty(dsa.dsa_masked_mha_workspace_size(mh.T_q, L_m), dtype=torch.uint8,
+                           device="cuda")
+
+        def mha_call():
+            dsa.dsa_masked_mha_fwd(mh.q, mh.k, mh.v, mh.idx, mh.cu_q, mh.cu_k, 1, L_m, L_m,
+                                   mh.topk, mh.scale, m_out, m_lse, workspace=m_ws, stream=stream)
+        for _ in range(3):
+            mha_call()
+        mev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(5)]
+        for e in mev:
+            flush.fill_(3.0)
+            e[0].record(stream)
+            mha_call()
+            e[1].record(stream)
+        torch.cuda.synchronize()
+        if dsa.dsa_get_device_error() != 0:
+            raise RuntimeError("device error in the masked MHA measurement")
+        m_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in mev]))
+        # dense causal attention: every (query, earlier key) pair of every head
+        m_flops = L_m * (L_m + 1) / 2 * 128 * 2 * (W.D_QK_MHA + W.D_V_MHA)
+        m_tf = m_flops / (m_ms / 1e3) / 1e12
+        mha_extra = {"workload": f"short prefill L={L_m}, H=128, d_qk=192, d_v=128, topk=2048",
+                     "ms": round(m_ms, 4), "bound": "tensor", "achieved": round(m_tf, 2),
+                     "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(m_tf / bf16_peak, 4),
+                     "work": "causal pairs x heads x 2*(192+128) flops",
+                     "traffic": ncu_traffic("masked_mha_kernel", f"mha-L{L_m}")}
+        del mh, m_out, m_lse, m_ws
+
     # ---- end to end through dsa_forward with host buffers
     e2e = None
     if not args.no_e2e and args.e2e_steps > 0:
@@ -388,6 +426,7 @@ def run_ours(args):
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": 3 * args.steps, "clocks": clk,
             "indexer_kl": kl_extra,
+            "masked_mha": mha_extra,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

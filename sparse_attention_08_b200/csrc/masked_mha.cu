@@ -19,16 +19,19 @@
 //  * masked_mha_kernel: one CTA per (tile of 128 queries of one sequence,
 //    head), flash-attention style over the causal key tiles of 128:
 //      warp 0  TMA: the query tile once (three 64-column boxes of a 3-D map
-//              [token, head, dim]), then key and value tiles into a two-stage
-//              ring;
+//              [token, head, dim]), then key tiles and value tiles into two
+//              two-stage rings of their own (a key stage frees when its S is
+//              done, a value stage after its P V);
 //      warp 1  TMEM owner and MMA issuer: S = Q K^T (12 tcgen05.mma, M = N =
 //              128, K = 16, both operands K-major in shared memory) into one
 //              of two S buffers, and O += P V (8 tcgen05.mma, P read from
 //              TMEM, V MN-major from shared memory);
-//      warps 2..5  one query row per thread (TMEM lane): masking (causal and
-//              the selection bits), online softmax in fp32 with a lazily
-//              rescaled maximum, P written to TMEM as bf16, and at the end O
-//              normalised and stored as bf16 together with the lse.
+//      warps 2..9  two warpgroups, one query row per thread (TMEM lane), each
+//              warpgroup half of the tile's keys and half of O's columns:
+//              masking (causal and the selection bits), online softmax in
+//              fp32 with a lazily rescaled maximum agreed between the halves,
+//              P written to TMEM as bf16, and at the end O normalised and
+//              stored as bf16 together with the lse.
 //    TMEM: S buffers at columns 0 and 128, P (128 x 128 bf16) at 256, O
 //    (128 x 128 fp32) at 320.
 #include <cuda_runtime.h>
@@ -47,15 +50,19 @@ constexpr int kDqk = 192;
 constexpr int kDv = 128;
 constexpr uint32_t kBox = 128 * 128;     // one 64-column box of 128 rows: 16 KB
 constexpr uint32_t kOffQ = 0;                          // 3 boxes
-constexpr uint32_t kOffKv = 3 * kBox;                  // stages of K (3 boxes) + V (2 boxes)
-constexpr uint32_t kStageBytes = 5 * kBox;             // 80 KB
 constexpr int kStages = 2;
-constexpr uint32_t kOffBar = kOffKv + kStages * kStageBytes;
-// barriers: q_full, kv_full[2], kv_empty[2], s_full[2], s_free[2], p_full, pv_done, drain
-constexpr uint32_t kNumBars = 1 + 2 * kStages + 4 + 3;
+constexpr uint32_t kOffK = 3 * kBox;                   // key stages: 3 boxes each
+constexpr uint32_t kKBytes = 3 * kBox;
+constexpr uint32_t kOffV = kOffK + kStages * kKBytes;  // value stages: 2 boxes each
+constexpr uint32_t kVBytes = 2 * kBox;
+constexpr uint32_t kOffBar = kOffV + kStages * kVBytes;
+// barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], s_free[2],
+// p_full, pv_done, drain
+constexpr uint32_t kNumBars = 1 + 4 * kStages + 4 + 3;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-constexpr uint32_t kSmem = kOffMisc + 16 + 1024;
-constexpr int kThreads = 192;
+constexpr uint32_t kOffXchg = kOffMisc + 16;           // row maxima and sums of the two halves
+constexpr uint32_t kSmem = kOffXchg + 1024 * 4 + 1024;
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;            // + 128 * buffer
 constexpr uint32_t kColP = 256;
@@ -130,13 +137,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + kOffBar;
   const uint32_t q_full = bar0;
-  auto kv_full = [&](uint32_t i) { return bar0 + 8u * (1 + i); };
-  auto kv_empty = [&](uint32_t i) { return bar0 + 8u * (1 + kStages + i); };
-  auto s_full = [&](uint32_t i) { return bar0 + 8u * (1 + 2 * kStages + i); };
-  auto s_free = [&](uint32_t i) { return bar0 + 8u * (3 + 2 * kStages + i); };
-  const uint32_t p_full = bar0 + 8u * (5 + 2 * kStages);
-  const uint32_t pv_done = bar0 + 8u * (6 + 2 * kStages);
-  const uint32_t drain = bar0 + 8u * (7 + 2 * kStages);
+  auto k_full = [&](uint32_t i) { return bar0 + 8u * (1 + i); };
+  auto k_empty = [&](uint32_t i) { return bar0 + 8u * (1 + kStages + i); };
+  auto v_full = [&](uint32_t i) { return bar0 + 8u * (1 + 2 * kStages + i); };
+  auto v_empty = [&](uint32_t i) { return bar0 + 8u * (1 + 3 * kStages + i); };
+  auto s_full = [&](uint32_t i) { return bar0 + 8u * (1 + 4 * kStages + i); };
+  auto s_free = [&](uint32_t i) { return bar0 + 8u * (3 + 4 * kStages + i); };
+  const uint32_t p_full = bar0 + 8u * (5 + 4 * kStages);
+  const uint32_t pv_done = bar0 + 8u * (6 + 4 * kStages);
+  const uint32_t drain = bar0 + 8u * (7 + 4 * kStages);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc);
 
   const int warp = threadIdx.x / 32;
@@ -159,14 +168,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(kv_full(i), 1);
-      mbar_init(kv_empty(i), 1);
+      mbar_init(k_full(i), 1);
+      mbar_init(k_empty(i), 1);
+      mbar_init(v_full(i), 1);
+      mbar_init(v_empty(i), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full(i), 1);
-      mbar_init(s_free(i), 4);
+      mbar_init(s_free(i), 8);
     }
-    mbar_init(p_full, 4);
+    mbar_init(p_full, 8);
     mbar_init(pv_done, 1);
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -182,42 +193,52 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA
+    // Lane 0 loads the query and the key tiles, lane 1 the value tiles: a key
+    // stage is free once its S product is done, a value stage only after its
+    // P V product, so the two rings run apart.
     if (lane == 0) {
       tma_prefetch_desc(&tq);
       tma_prefetch_desc(&tk);
-      tma_prefetch_desc(&tv);
       mbar_arrive_expect_tx(q_full, 3 * kBox);
       for (int c = 0; c < 3; ++c)
         tma_load_3d(sbase + kOffQ + c * kBox, &tq, 64 * c, h, cq0 + q0, q_full);
       for (int j = 0; j < n_tiles; ++j) {
         const uint32_t st = j & 1;
-        if (!mbar_wait(kv_empty(st), ((j >> 1) & 1) ^ 1, P.err)) break;
-        const uint32_t dst = sbase + kOffKv + st * kStageBytes;
-        const int row = ck0 + j * kBN;
-        mbar_arrive_expect_tx(kv_full(st), 5 * kBox);
-        for (int c = 0; c < 3; ++c) tma_load_3d(dst + c * kBox, &tk, 64 * c, h, row, kv_full(st));
+        if (!mbar_wait(k_empty(st), ((j >> 1) & 1) ^ 1, P.err)) break;
+        const uint32_t dst = sbase + kOffK + st * kKBytes;
+        mbar_arrive_expect_tx(k_full(st), kKBytes);
+        for (int c = 0; c < 3; ++c)
+          tma_load_3d(dst + c * kBox, &tk, 64 * c, h, ck0 + j * kBN, k_full(st));
+      }
+    } else if (lane == 1) {
+      tma_prefetch_desc(&tv);
+      for (int j = 0; j < n_tiles; ++j) {
+        const uint32_t st = j & 1;
+        if (!mbar_wait(v_empty(st), ((j >> 1) & 1) ^ 1, P.err)) break;
+        const uint32_t dst = sbase + kOffV + st * kVBytes;
+        mbar_arrive_expect_tx(v_full(st), kVBytes);
         for (int c = 0; c < 2; ++c)
-          tma_load_3d(dst + (3 + c) * kBox, &tv, 64 * c, h, row, kv_full(st));
+          tma_load_3d(dst + c * kBox, &tv, 64 * c, h, ck0 + j * kBN, v_full(st));
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA
     const uint64_t dQ = smem_desc(sbase + kOffQ, 16, 1024, kSwizzle128B);
-    const uint64_t dK0 = smem_desc(sbase + kOffKv, 16, 1024, kSwizzle128B);
-    const uint64_t dV0 = smem_desc(sbase + kOffKv + 3 * kBox, kBox, 1024, kSwizzle128B);
-    constexpr uint64_t kStageStep = kStageBytes >> 4;
+    const uint64_t dK0 = smem_desc(sbase + kOffK, 16, 1024, kSwizzle128B);
+    const uint64_t dV0 = smem_desc(sbase + kOffV, kBox, 1024, kSwizzle128B);
     bool ok = warp_wait(q_full, 0, P.err);
     auto issue_pv = [&](int j) -> bool {
-      if (!warp_wait(p_full, j & 1, P.err)) return false;
+      if (!warp_wait(p_full, j & 1, P.err) || !warp_wait(v_full(j & 1), (j >> 1) & 1, P.err))
+        return false;
       tc_fence_after();
-      const uint64_t dV = dV0 + (j & 1) * kStageStep;
+      const uint64_t dV = dV0 + (j & 1) * (kVBytes >> 4);
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
           mma_f16_ts(tmem + kColO, tmem + kColP + 8u * kk, dV + ((kk * 2048) >> 4), kIdescPV,
                      (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(kv_empty(j & 1));
+        mma_commit(v_empty(j & 1));
         mma_commit(pv_done);
       }
       __syncwarp();
@@ -225,11 +246,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     for (int j = 0; ok && j < n_tiles; ++j) {
       const uint32_t st = j & 1;
-      ok = warp_wait(kv_full(st), (j >> 1) & 1, P.err) &&
+      ok = warp_wait(k_full(st), (j >> 1) & 1, P.err) &&
            warp_wait(s_free(st), ((j >> 1) & 1) ^ 1, P.err);
       if (!ok) break;
       tc_fence_after();
-      const uint64_t dK = dK0 + st * kStageStep;
+      const uint64_t dK = dK0 + st * (kKBytes >> 4);
       if (elect_one()) {
 #pragma unroll
         for (int c = 0; c < 3; ++c) {
@@ -239,6 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     dK + ((c * kBox + kk * 32) >> 4), kIdescS, (c | kk) != 0 ? 1u : 0u);
         }
         mma_commit(s_full(st));
+        mma_commit(k_empty(st));
       }
       __syncwarp();
       if (j > 0) ok = issue_pv(j - 1);
@@ -249,42 +271,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
+    // Two warpgroups; warpgroup wg takes keys 64wg..64wg+63 of every tile
+    // (and the same 64 value dims of O), a thread one query row (TMEM lane).
+    // The halves meet once per tile to agree on the row maximum, through
+    // shared memory and a named barrier.
+    const int wg = (warp - 2) >> 2;                   // 0 or 1
     const int sp = warp & 3;                          // TMEM sub-partition
     const int r = sp * 32 + lane;                     // query row in the tile
     const uint32_t lane_base = static_cast<uint32_t>(sp * 32) << 16;
+    const uint32_t c0 = 64u * wg;                     // this half's first column
     const bool row_ok = r < rows;
     const int i = q0 + (row_ok ? r : rows - 1);       // local query index
-    const uint4* mrow = reinterpret_cast<const uint4*>(P.mask + static_cast<int64_t>(cq0 + i) * P.words);
+    const uint2* mrow = reinterpret_cast<const uint2*>(P.mask + static_cast<int64_t>(cq0 + i) * P.words);
+    float* pmax = reinterpret_cast<float*>(smem + kOffXchg);        // [2][2][128]
     float m = -INFINITY, l = 0.f, lr = 0.f;
     bool ok = true;
-    uint4 mw = __ldg(mrow);
+    bool bad = false;                                 // a wait of this warp gave up
+    uint2 mw = __ldg(mrow + wg);
     for (int j = 0; j < n_tiles; ++j) {
       const uint32_t st = j & 1;
-      if (!warp_wait(s_full(st), (j >> 1) & 1, P.err)) {
+      uint32_t v[64];
+      float mx = -INFINITY;
+      if (!bad) bad = !warp_wait(s_full(st), (j >> 1) & 1, P.err);
+      if (!bad) {
+        tc_fence_after();
+        tmem_ld_32x32b_x64(tmem + lane_base + kColS + 128u * st + c0, v);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free(st));
+        // mask: a key counts when it is selected (which implies s <= p) and
+        // the row exists; a warp whose 64 keys are all selected skips it
+        const uint32_t w0 = row_ok ? mw.x : 0u, w1 = row_ok ? mw.y : 0u;
+        if (j + 1 < n_tiles) mw = __ldg(mrow + 2 * (j + 1) + wg);
+        if (!__all_sync(0xffffffffu, (w0 & w1) == 0xffffffffu)) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (!(((c < 32 ? w0 : w1) >> (c & 31)) & 1u)) v[c] = 0xff800000u;
+        }
+#pragma unroll
+        for (int c = 0; c < 64; ++c) mx = fmaxf(mx, __uint_as_float(v[c]));
+      }
+      // the row maximum over both halves; the reducing barrier also takes
+      // both warpgroups out together when a wait of one of them gave up
+      float* px = pmax + st * 256;
+      px[wg * 128 + r] = mx;
+      if (named_bar_or(1, 256, bad)) {
         ok = false;
         break;
       }
-      tc_fence_after();
-      uint32_t v[128];
-      tmem_ld_32x32b_x64(tmem + lane_base + kColS + 128u * st, *reinterpret_cast<uint32_t(*)[64]>(v));
-      tmem_ld_32x32b_x64(tmem + lane_base + kColS + 128u * st + 64,
-                         *reinterpret_cast<uint32_t(*)[64]>(v + 64));
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free(st));
-      // mask: a key counts when it is selected (which implies s <= p) and the
-      // row exists
-      const uint32_t wd[4] = {row_ok ? mw.x : 0u, row_ok ? mw.y : 0u, row_ok ? mw.z : 0u,
-                              row_ok ? mw.w : 0u};
-      if (j + 1 < n_tiles) mw = __ldg(mrow + j + 1);
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        if (!((wd[c >> 5] >> (c & 31)) & 1u)) v[c] = 0xff800000u;
-        mx = fmaxf(mx, __uint_as_float(v[c]));
-      }
-      mx *= P.scale_log2;
+      mx = fmaxf(mx, px[(wg ^ 1) * 128 + r]) * P.scale_log2;
       float al = 1.f;
       bool moved = false;
       if (mx > m + kRescaleThreshold) {
@@ -293,52 +329,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         moved = true;
       }
       const float nm = m == -INFINITY ? 0.f : -m;
-      uint32_t pk[64];
-      float s_sum = 0.f, r_sum = 0.f;
+      const float2 sc2 = make_float2(P.scale_log2, P.scale_log2), nm2 = make_float2(nm, nm);
+      uint32_t pk[32];
+      float2 s2 = make_float2(0.f, 0.f), r2 = s2;
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = fast_exp2(fmaf(__uint_as_float(v[2 * c]), P.scale_log2, nm));
-        const float p1 = fast_exp2(fmaf(__uint_as_float(v[2 * c + 1]), P.scale_log2, nm));
-        s_sum += p0 + p1;
+      for (int c = 0; c < 32; ++c) {
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])),
+                                    sc2, nm2);
+        const float p0 = fast_exp2(x.x), p1 = fast_exp2(x.y);
+        s2 = __fadd2_rn(s2, make_float2(p0, p1));
         pk[c] = pack_bf16x2(p0, p1);
-        r_sum += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xFFFF0000u);
+        r2 = __fadd2_rn(r2, make_float2(__uint_as_float(pk[c] << 16), __uint_as_float(pk[c] & 0xFFFF0000u)));
       }
-      l = l * al + s_sum;
-      lr = lr * al + r_sum;
+      l = l * al + (s2.x + s2.y);
+      lr = lr * al + (r2.x + r2.y);
       // P and O are the previous P V's operands: wait until it is complete
       if (j > 0) {
         if (!warp_wait(pv_done, (j - 1) & 1, P.err)) {
-          ok = false;
-          break;
+          bad = true;                                 // the next barrier stops everyone
+          continue;
         }
         tc_fence_after();
         if (__any_sync(0xffffffffu, moved)) {
 #pragma unroll 1
-          for (int c = 0; c < kDv; c += 32) {
+          for (int c = 0; c < 64; c += 32) {
             uint32_t o[32];
-            tmem_ld_32x32b_x32(tmem + lane_base + kColO + c, o);
+            tmem_ld_32x32b_x32(tmem + lane_base + kColO + c0 + c, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * al);
-            tmem_st_32x32b_x32(tmem + lane_base + kColO + c, o);
+            tmem_st_32x32b_x32(tmem + lane_base + kColO + c0 + c, o);
           }
         }
       }
-      tmem_st_32x32b_x32(tmem + lane_base + kColP, *reinterpret_cast<uint32_t(*)[32]>(pk));
-      tmem_st_32x32b_x32(tmem + lane_base + kColP + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+      tmem_st_32x32b_x32(tmem + lane_base + kColP + 32u * wg, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    if (ok && warp_wait(pv_done, (n_tiles - 1) & 1, P.err)) {
+    // the two halves' sums (every thread reaches this exchange: a thread that
+    // stopped on a failed wait brings zeros and stores nothing)
+    float* px = pmax + 512;                           // [2][2][128]: l and lr per half
+    px[wg * 256 + r] = l;
+    px[wg * 256 + 128 + r] = lr;
+    named_bar_sync(1, 256);
+    const float l_all = l + px[(wg ^ 1) * 256 + r];
+    const float lr_all = lr + px[(wg ^ 1) * 256 + 128 + r];
+    if (ok && !bad && warp_wait(pv_done, (n_tiles - 1) & 1, P.err)) {
       tc_fence_after();
-      const float inv = lr > 0.f ? 1.f / lr : 0.f;
-      __nv_bfloat16* orow = P.out + (static_cast<int64_t>(cq0 + i) * P.H + h) * kDv;
+      const float inv = lr_all > 0.f ? 1.f / lr_all : 0.f;
+      __nv_bfloat16* orow = P.out + (static_cast<int64_t>(cq0 + i) * P.H + h) * kDv + c0;
 #pragma unroll 1
-      for (int c = 0; c < kDv; c += 32) {
+      for (int c = 0; c < 64; c += 32) {
         uint32_t o[32];
-        tmem_ld_32x32b_x32(tmem + lane_base + kColO + c, o);
+        tmem_ld_32x32b_x32(tmem + lane_base + kColO + c0 + c, o);
         tmem_wait_ld();
         if (row_ok) {
 #pragma unroll
@@ -352,9 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (row_ok && P.lse)
+      if (row_ok && wg == 0 && P.lse)
         P.lse[static_cast<int64_t>(cq0 + i) * P.H + h] =
-            l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+            l_all > 0.f ? (m + log2f(l_all)) * 0.69314718055994531f : -INFINITY;
     }
   }
 
