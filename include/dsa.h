@@ -235,8 +235,8 @@ DSA_API size_t dsa_forward_host_workspace_size(int64_t total_k, int max_len_k, i
 
 /*
  * The indexer's training signal ("DeepSeek V3.2 and the lightning indexer",
- * section "Teaching a dense model to be sparse": the indexer is trained with a
- * KL divergence loss to match the distribution of the main attention;
+ * section "Teaching a dense model to be sparse": the indexer's scores are
+ * fitted to the main attention's distribution by minimising a KL divergence;
  * "DeepSeek-V3.2" atlas entry, "Design overview": the target is the head-wise
  * attention distribution summed over heads).  For each query row t with valid
  * selected entries S (idx[t, j] with 0 <= idx <= p, j < min(k, p+1)):
@@ -271,8 +271,9 @@ DSA_API dsa_status_t dsa_indexer_kl(const void* q, const void* kv, const int32_t
 DSA_API size_t dsa_indexer_kl_workspace_size(int64_t total_q, int H, int k);
 
 /*
- * The masked MHA mode ("DeepSeek-V3.2" paper record: short-sequence
- * prefilling uses a masked MHA mode that simulates DSA; the pages give no
+ * The masked MHA mode ("DeepSeek-V3.2" atlas entry, "Design overview" and
+ * "Inference efficiency": short prompts are prefilled with a masked MHA
+ * standing in for DSA; the pages give no
  * detail, so it is read as dense attention in the MHA form of MLA -- per-head
  * keys and values -- restricted by a mask to each query's selected set):
  *

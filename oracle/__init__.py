@@ -16,7 +16,7 @@ indexer works"; "DeepSeek-V3.2" atlas entry, "Design overview"):
 * top-k    the min(k, p+1) best scores, ties to the lower index, ascending
 * attention softmax over the selected latents, shared by all query heads
 * masked MHA  dense per-head attention restricted to the selected set (the
-  short-prefill mode the "DeepSeek-V3.2" paper record names)
+  short-prefill mode the "DeepSeek-V3.2" atlas entry names in "Design overview")
 """
 from __future__ import annotations
 
@@ -284,8 +284,8 @@ def indexer_kl_at(q_bits, kv_bits, idx, pos, logits, scale):
 
 
 def masked_mha_at(q_bits, k_bits, v_bits, idx, pos, scale):
-    """The masked MHA mode ("DeepSeek-V3.2" paper record: short-sequence
-    prefilling uses a masked MHA mode that simulates DSA): per-head dense
+    """The masked MHA mode ("DeepSeek-V3.2" atlas entry, "Design overview":
+    short prompts are prefilled with a masked MHA standing in for DSA): per-head dense
     attention of query row r (position pos[r]) over the set of its valid
     selected keys.  q_bits [R, H, d_qk], k_bits [n_k, H, d_qk], v_bits
     [n_k, H, d_v] (bf16 bits), idx [R, topk].  Returns (out [R, H, d_v],

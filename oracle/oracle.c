@@ -411,8 +411,8 @@ int oracle_sparse_mla_at(const uint16_t* q, const uint16_t* kv, const int32_t* i
 
 /* KL alignment of the indexer to the main attention over the selected set
  * ("DeepSeek V3.2 and the lightning indexer", section "Teaching a dense model
- * to be sparse": the indexer is trained with a KL divergence loss to match
- * the distribution of the main attention; "DeepSeek-V3.2" atlas entry,
+ * to be sparse": the indexer's scores are fitted to the main attention's
+ * distribution by minimising a KL divergence; "DeepSeek-V3.2" atlas entry,
  * "Design overview": the target is the head-wise attention distribution
  * summed over heads).  Readings: the target of query row r over its valid
  * selected entries S (the index row's entries 0 <= s <= p) is
@@ -508,8 +508,8 @@ int oracle_indexer_kl_at(const uint16_t* q, const uint16_t* kv, const int32_t* i
 /* ---------------------------------------------------------------------- */
 
 /* The masked MHA mode that stands in for DSA on short prefills ("DeepSeek-
- * V3.2" paper record: short-sequence prefilling uses a masked MHA mode that
- * simulates DSA; the pages name it without detail).  Reading: dense attention
+ * V3.2" atlas entry, "Design overview" and "Inference efficiency" name it;
+ * the pages give no detail).  Reading: dense attention
  * in the MHA form of MLA (every head has its own key and value), restricted
  * by a mask to the query's selected set S = { idx[r, j] : 0 <= idx[r, j] <= p }
  * taken as a set (a repeated entry counts once), keys visited in ascending

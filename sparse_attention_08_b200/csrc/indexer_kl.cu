@@ -4,8 +4,8 @@
 // and its gradient with respect to those scores.
 //
 // What it computes ("DeepSeek V3.2 and the lightning indexer", section
-// "Teaching a dense model to be sparse": the indexer is trained with a KL
-// divergence loss to match the distribution of the main attention;
+// "Teaching a dense model to be sparse": the indexer's scores are fitted to
+// the main attention's distribution by minimising a KL divergence;
 // "DeepSeek-V3.2" atlas entry, "Design overview": the target is the head-wise
 // attention distribution summed over heads).  For query t with valid
 // selected entries S (index-row entries 0 <= s <= p):

@@ -1,8 +1,9 @@
 // masked_mha.cu -- the masked MHA mode on sm_100a.
 //
-// What it computes ("DeepSeek-V3.2" paper record: short-sequence prefilling
-// uses a masked MHA mode that simulates DSA; the pages name the mode without
-// detail, so it is read as dense attention in the MHA form of MLA -- every
+// What it computes ("DeepSeek-V3.2" atlas entry, "Design overview" and
+// "Inference efficiency": for short prompts the prefill runs a masked form of
+// MHA as a stand-in for DSA; the pages name the mode without detail, so it is
+// read as dense attention in the MHA form of MLA -- every
 // head with its own 192-d key (128 + 64 RoPE) and 128-d value -- restricted
 // by a mask to each query's selected set S_t):
 //

@@ -344,9 +344,10 @@ def make_small(H_I=4, d_I=64, H=16, L=300, k=64, seed=7, integer=False, device="
 
 
 # ---------------------------------------------------------------------------
-# Masked MHA mode ("DeepSeek-V3.2" paper record: short-sequence prefilling
-# uses a masked MHA mode that simulates DSA).  Per-head queries and keys of
-# 192 dims (128 + 64 RoPE) and values of 128 dims, the MHA form of MLA.
+# Masked MHA mode ("DeepSeek-V3.2" atlas entry, "Design overview" and
+# "Inference efficiency": for short prompts the prefill runs a masked form of
+# MHA as a stand-in for DSA).  Per-head queries and keys of 192 dims (128 + 64
+# RoPE) and values of 128 dims, the MHA form of MLA.
 
 D_QK_MHA = 192
 D_V_MHA = 128

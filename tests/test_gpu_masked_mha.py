@@ -1,5 +1,5 @@
-"""GPU parity of the masked MHA mode ("DeepSeek-V3.2" paper record: short-
-sequence prefilling uses a masked MHA mode that simulates DSA): the CUDA path
+"""GPU parity of the masked MHA mode ("DeepSeek-V3.2" atlas entry, "Design
+overview": short prompts are prefilled with a masked MHA standing in for DSA): the CUDA path
 through the C ABI against the fp64 oracle on the same seeded inputs.  Small
 cases are compared over every query row (several query and key tiles, ragged
 tails, varlen chunks); the benchmark's workload runs in the launch the

@@ -447,8 +447,9 @@ def test_kl_target_is_the_mean_of_the_single_head_targets_and_matches_attention(
 
 
 # ---------------------------------------------------------------------------
-# Masked MHA mode ("DeepSeek-V3.2" paper record: short-sequence prefilling
-# uses a masked MHA mode that simulates DSA).  Reading: dense per-head
+# Masked MHA mode ("DeepSeek-V3.2" atlas entry, "Design overview" and
+# "Inference efficiency": short prompts are prefilled with a masked MHA
+# standing in for DSA).  Reading: dense per-head
 # attention restricted to the selected set.
 
 def _mha_case(n=40, H=3, d_qk=24, d_v=8, seed=5):
