@@ -5,16 +5,17 @@
  *
  * The operation, as the pages state it:
  *  - "DeepSeek V3.2 and the lightning indexer" (montana-research blog),
- *    section "How the lightning indexer works": a few indexer heads score each
- *    query against every earlier token as a weighted sum of ReLU'd dot
- *    products, in FP8; each query keeps its 2,048 best entries; the main
- *    attention runs over those only; DSA sits on the MQA mode of MLA, so one
- *    latent serves all query heads and the selection is made per position.
+ *    section "How the lightning indexer works": the score of a query for an
+ *    earlier token adds up, over a handful of FP8 indexer heads, ReLU-clipped
+ *    dot products scaled by per-head weights; a query's 2,048 highest scores
+ *    pick the entries its attention reads, and nothing else; under MLA's MQA
+ *    form a latent is shared by all query heads, so one selection serves a
+ *    whole query position.
  *  - "DeepSeek-V3.2" (atlas.lewiswon.me), "Design overview": token-level
  *    top-k with k = 2048, main attention cost O(L*k).
- *  - "DeepSeek-V3.2 ... (introducing DSA)" (phantomic12 paper record): one
- *    scalar indexer logit per (query, KV) pair; only the top-k are attended;
- *    the indexer is a full-context pass, which is why it runs in FP8.
+ *  - "DeepSeek-V3.2 ... (introducing DSA)" (phantomic12 paper record): the
+ *    indexer gives each (query, KV) pair a single scalar and the attention
+ *    reads the k best; the indexer touches the whole context, hence FP8.
  *
  * Conventions shared by every call
  * --------------------------------

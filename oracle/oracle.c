@@ -13,20 +13,20 @@
  *
  * Sources (the pages this follows):
  *  - "DeepSeek V3.2 and the lightning indexer" (montana-research blog),
- *    section "How the lightning indexer works": the indexer score between a
- *    query and each earlier token is a weighted sum of ReLU-activated dot
- *    products computed by a few indexer heads, in FP8; the top 2,048 entries
- *    per query are kept and the main attention runs only over them; DSA runs on
- *    the MQA mode of MLA, so one selected latent is shared by every query head
- *    and the selection is made once per query position.
+ *    section "How the lightning indexer works": a handful of FP8 indexer heads
+ *    each take a ReLU-clipped dot product of the query with an earlier token,
+ *    and a per-head weight combines them into one score; a query keeps its
+ *    2,048 highest-scoring entries and its attention reads nothing else; under
+ *    MLA's MQA form every query head shares the selected latents, so there is
+ *    one selection per query position.
  *  - "DeepSeek-V3.2" (atlas.lewiswon.me), "Design overview" and the
  *    "Inference efficiency" row of the spec sheet: a few indexer heads score
  *    every query against all earlier tokens with ReLU and per-head weights;
  *    token-level top-k with k = 2048 per query; the main attention reads only
  *    the chosen latents.
- *  - "DeepSeek-V3.2 ... (introducing DSA)" (phantomic12 paper record): the FP8
- *    ReLU indexer yields one scalar logit per (query, KV) pair; only the top-k
- *    of those are attended.
+ *  - "DeepSeek-V3.2 ... (introducing DSA)" (phantomic12 paper record): each
+ *    (query, KV) pair gets a single scalar from the FP8 ReLU indexer, and the
+ *    attention reads the k best per query.
  *
  * Readings where the pages are silent:
  *  - causal: the query at absolute position p may use keys 0..p (self

@@ -1,8 +1,9 @@
 // indexer.cu -- lightning-indexer scores on sm_100a.
 //
 // What it computes ("DeepSeek V3.2 and the lightning indexer", section "How
-// the lightning indexer works": a few indexer heads score every query against
-// each earlier token as a weighted sum of ReLU'd dot products, in FP8):
+// the lightning indexer works": per query and earlier token, a handful of FP8
+// indexer heads each give a ReLU-clipped dot product, combined with per-head
+// weights into one score):
 //
 //   logits[t, s] = k_scale[s] * sum_j (w[t,j] * q_scale[t,j]) * ReLU(q8[t,j,:] . k8[s,:])
 //

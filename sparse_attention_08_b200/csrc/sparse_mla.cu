@@ -1,9 +1,8 @@
 // sparse_mla.cu -- sparse attention in the MQA mode of MLA on sm_100a.
 //
 // What it computes ("DeepSeek V3.2 and the lightning indexer", section "How
-// the lightning indexer works": the main attention runs only over the
-// selected entries, and in MQA mode every selected latent serves all query
-// heads; "DeepSeek-V3.2" atlas entry, "Inference efficiency": only the chosen
+// the lightning indexer works": attention reads nothing but the selected
+// entries, and in MQA mode each selected latent is used by every query head; "DeepSeek-V3.2" atlas entry, "Inference efficiency": only the chosen
 // latents of the cache are touched):
 //
 //   out[t,h,:] = sum_{s in S_t} softmax_s(scale * q[t,h,:] . c[s,:]) * c[s,0:512]
