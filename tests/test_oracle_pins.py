@@ -554,3 +554,24 @@ def test_masked_mha_is_the_mqa_mode_after_absorption():
     np.testing.assert_allclose(lse_mha, lse_mqa, rtol=1e-12, atol=1e-12)
     for h in range(H):
         np.testing.assert_allclose(out_mha[:, h], out_mqa[:, h] @ w_uv[h].T, rtol=1e-11, atol=1e-12)
+
+
+def test_masked_mha_inputs_follow_the_recipe():
+    """The masked-MHA workload's selection: per query at p, min(topk, p+1)
+    distinct keys of [0, p], ascending, then -1; every key when p+1 <= topk."""
+    m = W.make_mha([300, 200], [300, 40], H=2, topk=64, seed=11)
+    idx = m.idx.numpy()
+    row = 0
+    for lq, lk in zip(m.lens_q, m.lens_k):
+        for i in range(lq):
+            p = lk - lq + i
+            sel = idx[row + i]
+            n = min(m.topk, p + 1)
+            assert np.all(sel[n:] == -1)
+            s = sel[:n]
+            assert np.all(s >= 0) and np.all(s <= p) and np.all(np.diff(s) > 0)
+            if p + 1 <= m.topk:
+                assert np.array_equal(s, np.arange(p + 1))
+        row += lq
+    assert m.q.shape == (340, 2, 192) and m.k.shape == (500, 2, 192) and m.v.shape == (500, 2, 128)
+    assert abs(m.scale - 192 ** -0.5) < 1e-12
