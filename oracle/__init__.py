@@ -75,6 +75,8 @@ def _load():
         lib.oracle_indexer_kl_at.argtypes = [P, P, P, P, P, i64, i64, i64, i32, i32, i32,
                                              ctypes.c_double, P, P, P]
         lib.oracle_indexer_kl_at.restype = i32
+        lib.oracle_indexer_backward.restype = i32
+        lib.oracle_indexer_backward.argtypes = [P, P, P, P, P, i64, i64, i32, i32, P, P, P]
         lib.oracle_masked_mha_at.restype = i32
         lib.oracle_masked_mha_at.argtypes = [P, P, P, P, P, i64, i64, i32, i32, i32, i32,
                                              ctypes.c_double, P, P]
@@ -281,6 +283,32 @@ def indexer_kl_at(q_bits, kv_bits, idx, pos, logits, scale):
     if rc != 0:
         raise ValueError("oracle_indexer_kl_at: bad arguments")
     return kl, grad, target
+
+
+def indexer_backward(q_hat, w, k_hat, g, pos):
+    """The indexer's backward ("DeepSeek V3.2 and the lightning indexer",
+    "Teaching a dense model to be sparse": the warm-up trains the indexer
+    alone on the KL signal): for scores I[t,s] = sum_j w[t,j] *
+    ReLU(q_hat[t,j] . k_hat[s]) over s <= pos[t] and an upstream gradient g
+    [n_q, n_k] (dense; entries past pos[t] are ignored), returns (dq [n_q, H,
+    d], dw [n_q, H], dk [n_k, d]) in fp64; the ReLU's derivative is 0 at 0."""
+    q_hat = _c(q_hat, np.float64)
+    w = _c(w, np.float64)
+    k_hat = _c(k_hat, np.float64)
+    g = _c(g, np.float64)
+    pos = _c(pos, np.int64)
+    n_q, H, d = q_hat.shape
+    n_k = k_hat.shape[0]
+    if w.shape != (n_q, H) or k_hat.shape != (n_k, d) or g.shape != (n_q, n_k) or pos.shape != (n_q,):
+        raise ValueError("indexer_backward: shape mismatch")
+    dq = np.empty_like(q_hat)
+    dw = np.empty_like(w)
+    dk = np.empty_like(k_hat)
+    rc = _load().oracle_indexer_backward(_ptr(q_hat), _ptr(w), _ptr(k_hat), _ptr(g), _ptr(pos),
+                                         n_q, n_k, H, d, _ptr(dq), _ptr(dw), _ptr(dk))
+    if rc != 0:
+        raise ValueError("oracle_indexer_backward: bad arguments")
+    return dq, dw, dk
 
 
 def masked_mha_at(q_bits, k_bits, v_bits, idx, pos, scale):

@@ -503,6 +503,52 @@ int oracle_indexer_kl_at(const uint16_t* q, const uint16_t* kv, const int32_t* i
   return bad ? -1 : 0;
 }
 
+/* The indexer's backward ("DeepSeek V3.2 and the lightning indexer", section
+ * "Teaching a dense model to be sparse": in the dense warm-up only the
+ * indexer learns, from the KL signal above).  Given the gradient g of a loss
+ * with respect to the scores I[t,s] = sum_j w[t,j] * ReLU(q[t,j,:] . k[s,:])
+ * (s <= p_t; q and k the dequantized FP8 values), the chain rule gives
+ *     dw[t,j]   = sum_s g[t,s] * ReLU(q[t,j,:] . k[s,:])
+ *     dq[t,j,:] = sum_s g[t,s] * w[t,j] * [q[t,j,:] . k[s,:] > 0] * k[s,:]
+ *     dk[s,:]   = sum_t sum_j g[t,s] * w[t,j] * [q[t,j,:] . k[s,:] > 0] * q[t,j,:]
+ * with the ReLU's derivative taken as 0 at 0.  Row t of q, w and g is at
+ * position pos[t]; g is dense [n_q, n_k] and only s <= pos[t] is used.  q:
+ * n_q x H x d; w: n_q x H; k: n_k x d; outputs dq (n_q x H x d), dw
+ * (n_q x H), dk (n_k x d), all fp64.  dk sums over every row, so this runs
+ * serially over rows. */
+int oracle_indexer_backward(const double* q, const double* w, const double* k, const double* g,
+                            const int64_t* pos, int64_t n_q, int64_t n_k, int H, int d,
+                            double* dq, double* dw, double* dk) {
+  if (!q || !w || !k || !g || !pos || !dq || !dw || !dk || H <= 0 || d <= 0) return -1;
+  for (int64_t i = 0; i < n_q * H * d; ++i) dq[i] = 0.0;
+  for (int64_t i = 0; i < n_q * H; ++i) dw[i] = 0.0;
+  for (int64_t i = 0; i < n_k * d; ++i) dk[i] = 0.0;
+  for (int64_t t = 0; t < n_q; ++t) {
+    const int64_t p = pos[t];
+    if (p < 0 || p >= n_k) return -1;
+    for (int64_t s = 0; s <= p; ++s) {
+      const double gs = g[t * n_k + s];
+      if (gs == 0.0) continue;
+      const double* ks = k + s * d;
+      for (int j = 0; j < H; ++j) {
+        const double* qj = q + (t * H + j) * d;
+        double dot = 0.0;
+        for (int e = 0; e < d; ++e) dot += qj[e] * ks[e];
+        if (!(dot > 0.0)) continue;
+        dw[t * H + j] += gs * dot;
+        const double c = gs * w[t * H + j];
+        double* dqj = dq + (t * H + j) * d;
+        double* dks = dk + s * d;
+        for (int e = 0; e < d; ++e) {
+          dqj[e] += c * ks[e];
+          dks[e] += c * qj[e];
+        }
+      }
+    }
+  }
+  return 0;
+}
+
 /* ---------------------------------------------------------------------- */
 /* Masked MHA mode.                                                         */
 /* ---------------------------------------------------------------------- */

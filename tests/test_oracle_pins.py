@@ -575,3 +575,103 @@ def test_masked_mha_inputs_follow_the_recipe():
         row += lq
     assert m.q.shape == (340, 2, 192) and m.k.shape == (500, 2, 192) and m.v.shape == (500, 2, 128)
     assert abs(m.scale - 192 ** -0.5) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# The indexer's backward ("DeepSeek V3.2 and the lightning indexer",
+# "Teaching a dense model to be sparse": the warm-up trains the indexer alone
+# on the KL signal).
+
+def _backward_case(n_q=6, n_k=11, H=4, d=8, seed=21):
+    rng = np.random.default_rng(seed)
+    q = rng.normal(size=(n_q, H, d))
+    w = rng.normal(size=(n_q, H))
+    k = rng.normal(size=(n_k, d))
+    pos = np.sort(rng.choice(np.arange(n_k), size=n_q, replace=False))
+    g = rng.normal(size=(n_q, n_k))
+    return q, w, k, g, pos
+
+
+def test_indexer_backward_matches_torch_autograd():
+    """torch's autograd differentiates the score sum_t,s g[t,s] * I[t,s]; its
+    gradients are the backward for upstream g (ReLU'(0) = 0 in both)."""
+    q, w, k, g, pos = _backward_case()
+    dq, dw, dk = oracle.indexer_backward(q, w, k, g, pos)
+    qt = torch.tensor(q, requires_grad=True)
+    wt = torch.tensor(w, requires_grad=True)
+    kt = torch.tensor(k, requires_grad=True)
+    dots = torch.einsum("thd,sd->ths", qt, kt)
+    scores = torch.einsum("th,ths->ts", wt, torch.relu(dots))
+    causal = torch.arange(k.shape[0])[None, :] <= torch.tensor(pos)[:, None]
+    (scores * torch.tensor(g) * causal).sum().backward()
+    np.testing.assert_allclose(dq, qt.grad.numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dw, wt.grad.numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dk, kt.grad.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_indexer_backward_of_the_kl_loss_matches_finite_differences():
+    """Chained with the pinned KL oracle: the KL gradient with respect to the
+    scores, pushed through the backward, is the derivative of the KL loss with
+    respect to the indexer weights w (central differences; the loss recomputes
+    the scores from the perturbed weights)."""
+    q_t, kv_t, idx, pos_kl, _ = _kl_case(R=3, H=2, n_k=40, k=16, seed=5)
+    q_kl, kv_kl = _bits(q_t), _bits(kv_t)
+    R, n_k = idx.shape[0], 40
+    rng = np.random.default_rng(9)
+    H_I, d_I = 3, 6
+    qi = rng.normal(size=(R, H_I, d_I))
+    ki = rng.normal(size=(n_k, d_I))
+    wi = rng.normal(size=(R, H_I))
+
+    def scores(wv):
+        return np.einsum("tj,tjs->ts", wv, np.maximum(np.einsum("tjd,sd->tjs", qi, ki), 0.0))
+
+    def loss(wv):
+        kl, _, _ = oracle.indexer_kl_at(q_kl, kv_kl, idx, pos_kl,
+                                        scores(wv).astype(np.float32).astype(np.float64), 0.2)
+        return kl.sum()
+
+    # scores passed through float32 for the KL oracle's interface: use exactly
+    # representable weights so the rounding does not move them
+    wi = np.round(wi * 64) / 64
+    qi = np.round(qi * 16) / 16
+    ki = np.round(ki * 16) / 16
+    lg = scores(wi).astype(np.float32)
+    kl, grad, _ = oracle.indexer_kl_at(q_kl, kv_kl, idx, pos_kl, lg, 0.2)
+    g = np.zeros((R, n_k))
+    for r in range(R):
+        for j, s in enumerate(idx[r]):
+            if 0 <= s <= pos_kl[r]:
+                g[r, s] += grad[r, j]
+    _, dw, _ = oracle.indexer_backward(qi, wi, ki, g, pos_kl)
+    h = 2.0 ** -10
+    for t in range(R):
+        for j in range(H_I):
+            wp, wm = wi.copy(), wi.copy()
+            wp[t, j] += h
+            wm[t, j] -= h
+            fd = (loss(wp) - loss(wm)) / (2 * h)
+            assert abs(fd - dw[t, j]) <= 2e-3 * max(1.0, abs(dw[t, j])), (t, j, fd, dw[t, j])
+
+
+def test_indexer_backward_relu_gates_and_causality():
+    q, w, k, g, pos = _backward_case(seed=3)
+    # a key that every head scores negatively carries no gradient, and
+    # removing it changes nothing else
+    q[..., 0] = np.abs(q[..., 0]) + 0.1
+    k[0] = 0.0
+    k[0, 0] = -1.0
+    dq, dw, dk = oracle.indexer_backward(q, w, k, g, pos)
+    assert np.all(dk[0] == 0)
+    g0 = g.copy()
+    g0[:, 0] = 0.0
+    a = oracle.indexer_backward(q, w, k, g0, pos)
+    for x, y in zip((dq, dw, dk), a):
+        np.testing.assert_array_equal(x, y)
+    # entries of g past a row's position are ignored
+    g2 = g.copy()
+    for t, p in enumerate(pos):
+        g2[t, p + 1:] = 123.0
+    b = oracle.indexer_backward(q, w, k, g2, pos)
+    for x, y in zip((dq, dw, dk), b):
+        np.testing.assert_array_equal(x, y)
