@@ -15,6 +15,8 @@ indexer works"; "DeepSeek-V3.2" atlas entry, "Design overview"):
 * indexer  I[t,s] = sum_j w[t,j] * ReLU(qhat[t,j] . khat[s])  for s <= p
 * top-k    the min(k, p+1) best scores, ties to the lower index, ascending
 * attention softmax over the selected latents, shared by all query heads
+* indexer backward  the gradients in q_I, w and k_I of a gradient on the
+  scores (the warm-up trains the indexer alone)
 * masked MHA  dense per-head attention restricted to the selected set (the
   short-prefill mode the "DeepSeek-V3.2" atlas entry names in "Design overview")
 """
