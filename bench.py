@@ -10,7 +10,10 @@ Prints ONE JSON line on rank 0.  With --gpus N > 1 it runs under torchrun,
 one rank per GPU; every rank runs its own sequence (data-parallel, no
 collective on the data path) and the step time is the maximum over ranks.
 ``--impl reference`` times the CPU oracle (oracle/, fp64, host cores) on a
-bounded sample of the same workload.
+bounded sample of the same workload.  ``--split-sequence`` instead splits ONE
+sequence over the ranks (strong scaling): every rank holds a position shard
+of the key-side cache, gathers the whole cache with one all-gather per
+tensor, and runs its two zig-zag query blocks.
 """
 from __future__ import annotations
 
@@ -60,6 +63,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kl", action="store_true")
     ap.add_argument("--no-mha", action="store_true")
+    ap.add_argument("--split-sequence", action="store_true")
     return ap.parse_args()
 
 
@@ -482,6 +486,96 @@ def run_e2e(dsa, wl, args, world, local, stream):
 # reference arm: the CPU oracle
 # ---------------------------------------------------------------------------
 
+def run_split(args):
+    """One prefill split over the ranks by zig-zag query blocks (strong
+    scaling); the key-side cache arrives sharded by position and is gathered
+    inside the timed step."""
+    import sparse_attention_08_b200 as dsa
+    from sparse_attention_08_b200 import sharding as S
+    from sparse_attention_08_b200 import workloads as W
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dsa.load()
+    cfg = W.CONFIGS[args.config]
+    if cfg.decode or cfg.B != 1:
+        raise SystemExit("--split-sequence splits one prefill sequence")
+    wl = W.make_prefill(args.config, device="cuda", seed=W.seed_of(args.config))
+    L, H = wl.T_q, wl.q.shape[1]
+    k0, k1 = S.key_shard(L, world, rank)
+    shard = [wl.k8[k0:k1].clone(), wl.k_scale[k0:k1].clone(), wl.kv[k0:k1].clone()]
+    full = [torch.empty_like(wl.k8), torch.empty_like(wl.k_scale), torch.empty_like(wl.kv)]
+    blocks = S.zigzag_blocks(L, world, rank)
+    args_b = [S.block_args(q0, q1) for q0, q1 in blocks]
+    cus = [(torch.tensor(a["cu_q"], dtype=torch.int32, device="cuda"),
+            torch.tensor(a["cu_k"], dtype=torch.int32, device="cuda")) for a in args_b]
+    ws = torch.empty(max(dsa.dsa_forward_workspace_size(a["max_len_q"], a["max_len_k"], wl.k)
+                         for a in args_b), dtype=torch.uint8, device="cuda")
+    out = torch.empty((L, H, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((L, H), dtype=torch.float32, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        if world > 1:
+            for loc, dst in zip(shard, full):
+                dst.copy_(S.all_gather_rows(loc))
+        else:
+            for loc, dst in zip(shard, full):
+                dst.copy_(loc)
+        for a, (cq, ck) in zip(args_b, cus):
+            r, kr = a["q_rows"], a["key_rows"]
+            dsa.dsa_forward(wl.q8[r], wl.q_scale[r], wl.w[r], full[0][kr], full[1][kr], wl.q[r],
+                            full[2][kr], cq, ck, 1, a["max_len_q"], a["max_len_k"], wl.k, wl.scale,
+                            out[r], lse[r], ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier(device_ids=[local])
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    if dsa.dsa_get_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    if dsa.dsa_get_device_error() != 0:
+        raise RuntimeError("device error during the timed region")
+    step_ms = max_over_ranks(float(np.mean([e[0].elapsed_time(e[1]) for e in evs])))
+    value = L / (step_ms / 1e3)
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "fp8e4m3+bf16", "data": "synthetic",
+            "config": {"workload": f"{cfg.name} (one causal prefill split over the GPUs)",
+                       "L": L, "parallelism": f"zigzag{world}",
+                       "exchange": "one all-gather per key-side tensor inside the step",
+                       "l2": "flushed between steps (256 MiB write outside the timed events)"},
+            "gpu_launches": 3 * len(blocks) * args.steps, "clocks": clk}), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def run_reference(args):
     from sparse_attention_08_b200 import workloads as W
     world, rank, _ = dist_env()
@@ -519,6 +613,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.split_sequence:
+        run_split(args)
     else:
         run_ours(args)
 
