@@ -295,7 +295,8 @@ DSA_API size_t dsa_indexer_kl_workspace_size(int64_t total_q, int H, int k);
  *  lse      (device, nullable) f32 [total_q, H] (natural log)
  *  workspace (device) dsa_masked_mha_workspace_size bytes: the selection as a
  *           bitmask, rebuilt by every call
- *  Supported: d_qk = 192, d_v = 128, 1 <= H <= 65535, max_len_k <= 131072.
+ *  Supported: d_qk = 192, d_v = 128, 1 <= H <= 65535, 1 <= topk <= 131072,
+ *  max_len_k <= 131072.
  *  Arithmetic: bf16 tensor-core products, fp32 accumulation and softmax.
  */
 DSA_API dsa_status_t dsa_masked_mha_fwd(const void* q, const void* k, const void* v,
