@@ -64,7 +64,7 @@ extern "C" {
 typedef enum {
   DSA_OK = 0,
   DSA_ERR_INVALID_ARG = 1, /* a size, count or pointer is out of range / NULL */
-  DSA_ERR_UNSUPPORTED = 2, /* valid but outside the shapes this build supports */
+  DSA_ERR_UNSUPPORTED = 2, /* valid but outside the shapes the library supports */
   DSA_ERR_ALIGNMENT = 3,   /* a pointer or stride breaks the 16-byte rule */
   DSA_ERR_WORKSPACE = 4,   /* workspace NULL or smaller than required */
   DSA_ERR_CUDA = 5,        /* a CUDA runtime / driver call failed */
