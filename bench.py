@@ -36,7 +36,17 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "DSA query-tokens/s (indexer+top-2048+sparse MLA) at L=32K; % roofline"
+METRICS = {
+    0: "DSA query-tokens/s (indexer+top-128+sparse MLA, 16 heads) at L=1K; % roofline",
+    1: "DSA query-tokens/s (indexer+top-2048+sparse MLA) at L=8K; % roofline",
+    2: METRIC,
+    3: "DSA query-tokens/s (indexer+top-2048+sparse MLA), decode batch of 64 over 4K-131K "
+       "caches; % roofline",
+    4: "DSA query-tokens/s (indexer+top-2048+sparse MLA), L=128K prefill in 8 chunks of 16K; "
+       "% roofline",
+}
 UNIT = "query-tokens/s"
+EXTRA_CONFIGS = (1, 3, 4)      # measured beside the headline on the default line
 L2_FLUSH_BYTES = 256 << 20
 KERNEL_FILES = {
     "indexer_kernel": "sparse_attention_08_b200/csrc/indexer.cu",
@@ -64,6 +74,8 @@ def parse_args():
     ap.add_argument("--no-kl", action="store_true")
     ap.add_argument("--no-mha", action="store_true")
     ap.add_argument("--split-sequence", action="store_true")
+    ap.add_argument("--no-extra-configs", action="store_true",
+                    help="measure only --config, not the other full-size configs")
     return ap.parse_args()
 
 
@@ -128,24 +140,66 @@ def ncu_traffic(kernel, workload):
 
 
 def counts(wl):
-    """Algorithmic work of one pass over the workload."""
-    causal, attended = 0, 0
+    """Algorithmic work of one pass over the workload (one call of each stage):
+    flops on the tensor cores and the bytes that must cross HBM at least once."""
+    causal, attended, lat_rows = 0, 0, 0
     for nq, nk in zip(wl.lens_q, wl.lens_k):
         causal += nq * (nk - nq) + nq * (nq + 1) // 2
         for i in range(nq):
             attended += min(wl.k, nk - nq + i + 1)
+        # distinct latent rows the sequence's selections can touch
+        lat_rows += min(nk, nq * wl.k)
     H_I, d_I = wl.q8.shape[1], wl.q8.shape[2]
     H = wl.q.shape[1]
+    T_q, T_k = wl.T_q, wl.T_k
     return {
         "causal_pairs": causal,
         "attended_pairs": attended,
         # FP8 products of the indexer contraction (2 flops per MAC)
         "indexer_flops": 2 * H_I * d_I * causal,
+        # indexer queries, weights and scales in; keys and their scales in
+        # once; every causal score written once
+        "indexer_bytes": T_q * H_I * (d_I + 8) + T_k * (d_I + 4) + 4 * causal,
+        "topk_flops": 0,
+        # top-k: read every causal score once, write k indices per query
+        "topk_bytes": 4 * causal + 4 * wl.k * T_q,
         # QK^T over 576 dims + PV over 512 dims for every head and attended pair
         "attention_flops": attended * H * (2 * 576 + 2 * 512),
-        # top-k: read every causal score once, write k indices per query
-        "topk_bytes": 4 * causal + 4 * wl.k * sum(wl.lens_q),
+        # queries in, outputs and lse out, indices in, every distinct latent
+        # row the selections touch once (L2 serves the repeats)
+        "attention_bytes": (T_q * H * (576 + 512) * 2 + T_q * H * 4 + 4 * wl.k * T_q
+                            + lat_rows * 576 * 2),
     }
+
+
+def add_counts(a, b):
+    return {n: a[n] + b[n] for n in a}
+
+
+def stage_rooflines(c, stage_ms, peaks):
+    """Per stage: the bound is whichever of (tensor flops / tensor peak) and
+    (HBM bytes / HBM bandwidth) takes longer; achieved is the work of that
+    bound over the measured time.  Peaks are the burst figures (the kernels
+    run at 1.8-1.97 GHz, as the cuBLAS burst did), FP8 at twice bf16."""
+    tens = {"indexer_kernel": 2.0 * peaks["bf16_tflops"], "topk_kernel": None,
+            "sparse_mla_kernel": peaks["bf16_tflops"]}
+    keys = {"indexer_kernel": "indexer", "topk_kernel": "topk",
+            "sparse_mla_kernel": "attention"}
+    out, t_roof = {}, 0.0
+    for i, n in enumerate(("indexer_kernel", "topk_kernel", "sparse_mla_kernel")):
+        fl, by = c[keys[n] + "_flops"], c[keys[n] + "_bytes"]
+        t_t = fl / (tens[n] * 1e12) if tens[n] else 0.0
+        t_m = by / (peaks["hbm_gbs"] * 1e9)
+        ms = float(stage_ms[i])
+        if t_t >= t_m:
+            ach, peak, unit, bound = fl / (ms / 1e3) / 1e12, tens[n], "TFLOP/s", "tensor"
+        else:
+            ach, peak, unit, bound = by / (ms / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
+        t_roof += max(t_t, t_m)
+        out[n] = {"ms": round(ms, 4), "bound": bound, "achieved": round(ach, 2),
+                  "peak": peak, "unit": unit, "frac": round(ach / peak, 4),
+                  "roof_ms": round(max(t_t, t_m) * 1e3, 4)}
+    return out, t_roof
 
 
 class ClockSampler:
@@ -204,23 +258,54 @@ class ClockSampler:
 # CPU oracle timing (reference arm and cpu_baseline)
 # ---------------------------------------------------------------------------
 
+def oracle_rows(L, k, n_rows, seed):
+    """A stratified sample of positions of one causal prefill of length L:
+    the edge positions 0, k-1, k and L-1, and one position drawn uniformly
+    from each of the remaining equal-width strata of [0, L)."""
+    rng = np.random.default_rng(seed)
+    fixed = sorted({p for p in (0, k - 1, k, L - 1) if 0 <= p < L})
+    m = max(0, n_rows - len(fixed))
+    edges = np.linspace(0, L, m + 1)
+    drawn = [int(rng.integers(int(edges[i]), max(int(edges[i]) + 1, int(edges[i + 1]))))
+             for i in range(m)]
+    return np.array(sorted(set(fixed) | set(drawn)), dtype=np.int64)
+
+
+def oracle_row_cost(p, k, H_I, d_I, H):
+    """Per-row work of the oracle at position p: p+1 indexer pairs and
+    min(p+1, k) attended pairs, in flops."""
+    p = np.asarray(p, dtype=np.float64)
+    return (p + 1) * 2 * H_I * d_I + np.minimum(p + 1, k) * H * (2 * 576 + 2 * 512)
+
+
 def oracle_sample(wl, n_rows, seed):
-    """Runs the oracle on n_rows query rows drawn uniformly over positions (all
-    host cores, one OpenMP region); returns (elapsed seconds, description)."""
+    """Runs the oracle (all host cores, one OpenMP region) on a stratified
+    sample of the query rows of a one-sequence prefill and extrapolates the
+    time of the whole workload with the per-row cost model.  Returns (sample
+    seconds, extrapolated query-tokens/s, description)."""
     import oracle
     from tests import dsa_cases as C
-    rng = np.random.default_rng(seed)
-    rows = np.sort(rng.choice(wl.T_q, size=n_rows, replace=False)).astype(np.int64)
     n_k = wl.lens_k[0]
+    L = wl.T_q
+    rows = oracle_rows(L, wl.k, n_rows, seed)
     k8, ks, kvb = C.np_(wl.k8[:n_k]), C.np_(wl.k_scale[:n_k]), C.bits(wl.kv[:n_k])
     rt = torch.as_tensor(rows, device=wl.q8.device)
     q8, qs, w = C.np_(wl.q8[rt]), C.np_(wl.q_scale[rt]), C.np_(wl.w[rt])
     qb = C.bits(wl.q[rt])
-    pos = rows + (n_k - wl.T_q)
+    pos = rows + (n_k - L)
     t0 = time.perf_counter()
     oracle.forward_at(q8, qs, w, k8, ks, qb, kvb, pos, wl.k, wl.scale)
     dt = time.perf_counter() - t0
-    return dt, f"{n_rows} query rows drawn uniformly over positions 0..{wl.T_q - 1}"
+    H_I, d_I, H = wl.q8.shape[1], wl.q8.shape[2], wl.q.shape[1]
+    all_pos = np.arange(n_k - L, n_k)
+    full = float(oracle_row_cost(all_pos, wl.k, H_I, d_I, H).sum())
+    part = float(oracle_row_cost(pos, wl.k, H_I, d_I, H).sum())
+    full_s = dt * full / part
+    desc = (f"{len(rows)} query rows, stratified over positions 0..{L - 1} (0, k-1, k, L-1 "
+            f"and one per stratum); the whole workload's time extrapolated from the sample by "
+            f"the per-row flop model (p+1 indexer pairs, min(p+1,k) attended pairs): "
+            f"{full_s:.0f} s")
+    return dt, L / full_s, desc
 
 
 def oracle_threads():
@@ -230,6 +315,104 @@ def oracle_threads():
 # ---------------------------------------------------------------------------
 # our implementation
 # ---------------------------------------------------------------------------
+
+def make_workload(cfg_id, seed):
+    from sparse_attention_08_b200 import workloads as W
+    if W.CONFIGS[cfg_id].decode:
+        return W.make_decode(cfg_id, device="cuda", seed=seed)
+    return W.make_prefill(cfg_id, device="cuda", seed=seed)
+
+
+class Stepper:
+    """One step of the path over a workload: the three stages on one stream,
+    once per chunk of a chunked prefill (each chunk's queries against the
+    cache up to its end), else once over the whole batch."""
+
+    def __init__(self, dsa, wl, stream):
+        from sparse_attention_08_b200 import workloads as W
+        self.dsa, self.wl, self.stream = dsa, wl, stream
+        if wl.cfg.chunks > 1:
+            C = wl.T_q // wl.cfg.chunks
+            self.parts = [(c * C, W.chunk_of(wl, c, C)) for c in range(wl.cfg.chunks)]
+        else:
+            self.parts = [(0, wl)]
+        H = wl.q.shape[1]
+        self.ld = (wl.max_len_k + 3) // 4 * 4
+        rows = max(p.T_q for _, p in self.parts)
+        self.logits = torch.empty((rows, self.ld), dtype=torch.float32, device="cuda")
+        self.idx = torch.empty((wl.T_q, wl.k), dtype=torch.int32, device="cuda")
+        self.out = torch.empty((wl.T_q, H, 512), dtype=torch.bfloat16, device="cuda")
+        self.lse = torch.empty((wl.T_q, H), dtype=torch.float32, device="cuda")
+
+    def launches(self):
+        return 3 * len(self.parts)
+
+    def step(self, ev=None):
+        """ev: None, or per part a list of 4 events around the three stages."""
+        dsa, s = self.dsa, self.stream
+        for pi, (r0, p) in enumerate(self.parts):
+            e = ev[pi] if ev is not None else None
+            r1 = r0 + p.T_q
+            if e is not None:
+                e[0].record(s)
+            dsa.dsa_indexer_logits(p.q8, p.q_scale, p.w, p.k8, p.k_scale, p.cu_q, p.cu_k, p.B,
+                                   p.max_len_q, p.max_len_k, self.logits, self.ld, stream=s)
+            if e is not None:
+                e[1].record(s)
+            dsa.dsa_topk(self.logits, p.cu_q, p.cu_k, p.B, p.max_len_q, p.max_len_k, p.k,
+                         self.idx[r0:r1], ld_logits=self.ld, stream=s)
+            if e is not None:
+                e[2].record(s)
+            dsa.dsa_sparse_mla_fwd(p.q, p.kv, self.idx[r0:r1], p.cu_q, p.cu_k, p.B, p.max_len_q,
+                                   p.max_len_k, p.scale, self.out[r0:r1], self.lse[r0:r1],
+                                   stream=s)
+            if e is not None:
+                e[3].record(s)
+
+    def counts(self):
+        c = None
+        for _, p in self.parts:
+            c = counts(p) if c is None else add_counts(c, counts(p))
+        return c
+
+
+def measure(dsa, st, steps, warmup, flush, clocks=None, barrier=None):
+    """Warm-up, then `steps` timed steps with L2 flushed before each (outside
+    the events).  Returns (mean ms per step, mean ms per stage [3], clocks)."""
+    for _ in range(warmup):
+        flush.fill_(1.0)
+        st.step()
+    torch.cuda.synchronize()
+    if dsa.dsa_get_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+    n = len(st.parts)
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+           for _ in range(steps)]
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+    for i in range(steps):
+        flush.fill_(float(i))           # evicts L2 between steps (outside the events)
+        st.step(evs[i])
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    clk = clocks.stop() if clocks else None
+    if dsa.dsa_get_device_error() != 0:
+        raise RuntimeError("device error during the timed region")
+    per = np.array([[sum(evs[i][pi][j].elapsed_time(evs[i][pi][j + 1]) for pi in range(n))
+                     for j in range(3)] for i in range(steps)])      # ms per stage per step
+    return float(per.sum(axis=1).mean()), per.mean(axis=0), clk
+
+
+def config_line(cfg_id, st, step_ms, stage_ms, peaks, world):
+    """Throughput and rooflines of one measured configuration."""
+    c = st.counts()
+    stages, t_roof = stage_rooflines(c, stage_ms, peaks)
+    return c, stages, t_roof, aggregate_value(world, st.wl.T_q, step_ms)
+
 
 def run_ours(args):
     import sparse_attention_08_b200 as dsa
@@ -243,112 +426,54 @@ def run_ours(args):
     dsa.load()
     cfg = W.CONFIGS[args.config]
     seed = rank_seed(args.config, rank)
-    if cfg.decode:
-        # a varlen decode batch (not the headline; a measurement of that shape)
-        wl = W.make_decode(args.config, device="cuda", seed=seed)
-    else:
-        wl = W.make_prefill(args.config, device="cuda", seed=seed)
+    wl = make_workload(args.config, seed)
+    st = Stepper(dsa, wl, torch.cuda.current_stream())
     H_I, d_I, H = wl.q8.shape[1], wl.q8.shape[2], wl.q.shape[1]
-    ld = (wl.max_len_k + 3) // 4 * 4
-    logits = torch.empty((wl.T_q, ld), dtype=torch.float32, device="cuda")
-    idx = torch.empty((wl.T_q, wl.k), dtype=torch.int32, device="cuda")
-    out = torch.empty((wl.T_q, H, 512), dtype=torch.bfloat16, device="cuda")
-    lse = torch.empty((wl.T_q, H), dtype=torch.float32, device="cuda")
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
-    stream = torch.cuda.current_stream()
-
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        dsa.dsa_indexer_logits(wl.q8, wl.q_scale, wl.w, wl.k8, wl.k_scale, wl.cu_q, wl.cu_k, wl.B,
-                               wl.max_len_q, wl.max_len_k, logits, ld, stream=stream)
-        if ev is not None:
-            ev[1].record(stream)
-        dsa.dsa_topk(logits, wl.cu_q, wl.cu_k, wl.B, wl.max_len_q, wl.max_len_k, wl.k, idx,
-                     ld_logits=ld, stream=stream)
-        if ev is not None:
-            ev[2].record(stream)
-        dsa.dsa_sparse_mla_fwd(wl.q, wl.kv, idx, wl.cu_q, wl.cu_k, wl.B, wl.max_len_q,
-                               wl.max_len_k, wl.scale, out, lse, stream=stream)
-        if ev is not None:
-            ev[3].record(stream)
-
-    for _ in range(args.warmup):
-        flush.fill_(1.0)
-        step()
-    torch.cuda.synchronize()
-    if dsa.dsa_get_device_error() != 0:
-        raise RuntimeError("device error during warm-up")
+    stream = st.stream
 
     def barrier():
         if world > 1:
             import torch.distributed as dist
             dist.barrier(device_ids=[local])
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    clocks = ClockSampler(local)
-    barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    for i in range(args.steps):
-        flush.fill_(float(i))           # evicts L2 between steps (outside the events)
-        step(evs[i])
-    torch.cuda.synchronize()
-    barrier()
-    clk = clocks.stop()
-    if dsa.dsa_get_device_error() != 0:
-        raise RuntimeError("device error during the timed region")
-    st = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)]
-                   for i in range(args.steps)])             # ms per stage per step
-    step_ms = float(st.sum(axis=1).mean())
-    stage_ms = st.mean(axis=0)
+    step_ms, stage_ms, clk = measure(dsa, st, args.steps, args.warmup, flush,
+                                     clocks=ClockSampler(local), barrier=barrier)
     step_ms = max_over_ranks(step_ms)
-    value = aggregate_value(world, wl.T_q, step_ms)
+    peaks = measured_peaks()
+    c, stages, t_roof, value = config_line(args.config, st, step_ms, stage_ms, peaks, world)
 
     # ---- roofline of the dominant kernel and of the whole step
-    peaks = measured_peaks()
-    c = counts(wl)
-    fp8_peak = 2.0 * peaks["bf16_tflops_sustained"]     # nominal fp8:bf16 ratio 2
-    bf16_peak = peaks["bf16_tflops_sustained"]
     names = ("indexer_kernel", "topk_kernel", "sparse_mla_kernel")
-    per = {
-        "indexer_kernel": ("tensor", c["indexer_flops"] / (stage_ms[0] / 1e3) / 1e12, fp8_peak,
-                           "TFLOP/s"),
-        "topk_kernel": ("hbm", c["topk_bytes"] / (stage_ms[1] / 1e3) / 1e9, peaks["hbm_gbs"],
-                        "GB/s"),
-        "sparse_mla_kernel": ("tensor", c["attention_flops"] / (stage_ms[2] / 1e3) / 1e12,
-                              bf16_peak, "TFLOP/s"),
-    }
     dom = names[int(np.argmax(stage_ms))]
-    bound, ach, peak, unit = per[dom]
-    workload_name = f"{cfg.name}"
-    roofline = {"kernel": dom, "bound": bound, "achieved": round(ach, 2), "peak": peak,
-                "unit": unit, "frac": round(ach / peak, 4),
-                "traffic": ncu_traffic(dom, workload_name),
-                "peak_source": f"{peaks['source']} (sustained bf16" +
-                               (", x2 for fp8)" if dom == "indexer_kernel" else ")")}
-    t_roof = (c["indexer_flops"] / (fp8_peak * 1e12) + c["topk_bytes"] / (peaks["hbm_gbs"] * 1e9)
-              + c["attention_flops"] / (bf16_peak * 1e12))
-    roofline["step_frac"] = round(t_roof * 1e3 / step_ms, 4)
-    roofline["stages"] = {n: {"ms": round(float(stage_ms[i]), 4), "bound": per[n][0],
-                              "achieved": round(per[n][1], 2), "peak": per[n][2],
-                              "unit": per[n][3], "frac": round(per[n][1] / per[n][2], 4)}
-                          for i, n in enumerate(names)}
+    d = stages[dom]
+    sustained = peaks["bf16_tflops_sustained"]
+    roofline = {"kernel": dom, "bound": d["bound"], "achieved": d["achieved"],
+                "peak": d["peak"], "unit": d["unit"], "frac": d["frac"],
+                "traffic": ncu_traffic(dom, cfg.name) if len(st.parts) == 1 else None,
+                "peak_source": f"{peaks['source']}: burst bf16 (x2 for fp8) and HBM copy",
+                "step_frac": round(t_roof * 1e3 / step_ms, 4),
+                "step_roof_ms": round(t_roof * 1e3, 4),
+                "stages": stages}
+    if d["unit"] == "TFLOP/s":
+        roofline["frac_of_sustained"] = round(
+            d["achieved"] / (sustained * (2.0 if dom == "indexer_kernel" else 1.0)), 4)
 
     # ---- the indexer's KL training signal on the same workload (not part of
     # the step): its score products are the attention's S half, M = 128
     kl_extra = None
-    if not args.no_kl and world == 1:
+    bf16_peak = peaks["bf16_tflops"]
+    if not args.no_kl and world == 1 and len(st.parts) == 1:
         kl = torch.empty((wl.T_q,), dtype=torch.float32, device="cuda")
         grad = torch.empty((wl.T_q, wl.k), dtype=torch.float32, device="cuda")
         ws_kl = torch.empty(max(16, dsa.dsa_indexer_kl_workspace_size(wl.T_q, H, wl.k)),
                             dtype=torch.uint8, device="cuda")
 
         def kl_call():
-            dsa.dsa_indexer_kl(wl.q, wl.kv, idx, lse, logits, wl.cu_q, wl.cu_k, wl.B,
+            dsa.dsa_indexer_kl(wl.q, wl.kv, st.idx, st.lse, st.logits, wl.cu_q, wl.cu_k, wl.B,
                                wl.max_len_q, wl.max_len_k, wl.k, wl.scale, kl, grad,
-                               workspace=ws_kl, ld_logits=ld, stream=stream)
-        for _ in range(2):
+                               workspace=ws_kl, ld_logits=st.ld, stream=stream)
+        for _ in range(3):
             kl_call()
         kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(3)]
         for e in kev:
@@ -361,9 +486,9 @@ def run_ours(args):
             raise RuntimeError("device error in the KL measurement")
         kl_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in kev]))
         s_flops = c["attended_pairs"] * H * 2 * 576
-        kl_extra = {"ms": round(kl_ms, 4), "bound": "tensor",
-                    "achieved": round(s_flops / (kl_ms / 1e3) / 1e12, 2), "peak": bf16_peak,
-                    "unit": "TFLOP/s", "frac": round(s_flops / (kl_ms / 1e3) / 1e12 / bf16_peak, 4),
+        kl_tf = s_flops / (kl_ms / 1e3) / 1e12
+        kl_extra = {"ms": round(kl_ms, 4), "bound": "tensor", "achieved": round(kl_tf, 2),
+                    "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(kl_tf / bf16_peak, 4),
                     "work": "S = Q K^T of every head and selected entry (2*576 flops each)",
                     "traffic": ncu_traffic("attn_target_kernel", f"{cfg.name}")}
         del ws_kl, grad
@@ -404,34 +529,62 @@ def run_ours(args):
                      "traffic": ncu_traffic("masked_mha_kernel", f"mha-L{L_m}")}
         del mh, m_out, m_lse, m_ws
 
-    # ---- end to end through dsa_forward with host buffers
+    # ---- end to end through the host-buffer entry point
     e2e = None
-    if not args.no_e2e and args.e2e_steps > 0:
+    if not args.no_e2e and args.e2e_steps > 0 and len(st.parts) == 1:
         e2e = run_e2e(dsa, wl, args, world, local, stream)
 
     # ---- CPU baseline: the oracle, rank 0 at N=1 only
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline and not cfg.decode:
-        n_rows = max(8, min(64, 2 * oracle_threads()))
-        dt, desc = oracle_sample(wl, n_rows, seed=99)
-        cpu = {"value": round(n_rows / dt, 4), "unit": UNIT, "cores": oracle_threads(),
-               "kind": "oracle", "sample": desc, "seconds": round(dt, 2)}
+        n_rows = max(20, min(64, 2 * oracle_threads()))
+        dt, v, desc = oracle_sample(wl, n_rows, seed=99)
+        cpu = {"value": round(v, 4), "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+               "sample": desc, "seconds": round(dt, 2)}
+
+    line = {
+        "metric": METRICS[args.config], "value": round(value, 1), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8e4m3+bf16", "data": "synthetic",
+        "config": {"workload": f"{cfg.name} (" + ("one varlen decode batch" if cfg.decode else
+                                                  "one causal prefill") + " per GPU)",
+                   "L": cfg.L, "H_I": H_I, "d_I": d_I, "H": H, "d_qk": 576, "d_v": 512,
+                   "k": wl.k, "chunks": cfg.chunks, "global_batch_sequences": world * wl.B,
+                   "parallelism": f"dp{world}",
+                   "l2": "flushed between steps (256 MiB write outside the timed events)"},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": st.launches() * args.steps, "clocks": clk,
+        "indexer_kl": kl_extra,
+        "masked_mha": mha_extra,
+    }
+    del st, wl
+
+    # ---- the other full-size configurations at one GPU, each with its own
+    # metric and per-stage rooflines (fewer timed steps; same timing rules)
+    if world == 1 and not args.no_extra_configs:
+        extra = {}
+        for cid in EXTRA_CONFIGS:
+            if cid == args.config:
+                continue
+            torch.cuda.empty_cache()
+            xw = make_workload(cid, rank_seed(cid, rank))
+            xs = Stepper(dsa, xw, stream)
+            x_steps = max(3, min(args.steps, 5))
+            xms, xstage, xclk = measure(dsa, xs, x_steps, 3, flush, clocks=ClockSampler(local))
+            xc, xstages, xroof, xval = config_line(cid, xs, xms, xstage, peaks, 1)
+            xcfg = W.CONFIGS[cid]
+            extra[xcfg.name] = {
+                "metric": METRICS[cid], "value": round(xval, 1), "unit": UNIT,
+                "ms_per_step": round(xms, 4), "steps": x_steps, "warmup": 3,
+                "queries_per_step": xw.T_q, "chunks": xcfg.chunks,
+                "step_frac": round(xroof * 1e3 / xms, 4), "step_roof_ms": round(xroof * 1e3, 4),
+                "stages": xstages, "gpu_launches": xs.launches() * x_steps, "clocks": xclk}
+            del xs, xw
+        line["configs"] = extra
+        line["gpu_launches"] += sum(v["gpu_launches"] for v in extra.values())
 
     if rank == 0:
-        line = {
-            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "fp8e4m3+bf16", "data": "synthetic",
-            "config": {"workload": f"{cfg.name} (" + ("one varlen decode batch" if cfg.decode else "one causal prefill") + " per GPU)", "L": cfg.L,
-                       "H_I": H_I, "d_I": d_I, "H": H, "d_qk": 576, "d_v": 512, "k": wl.k,
-                       "global_batch_sequences": world, "parallelism": f"dp{world}",
-                       "l2": "flushed between steps (256 MiB write outside the timed events)"},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": 3 * args.steps, "clocks": clk,
-            "indexer_kl": kl_extra,
-            "masked_mha": mha_extra,
-        }
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -562,7 +715,7 @@ def run_split(args):
     value = L / (step_ms / 1e3)
     if rank == 0:
         print(json.dumps({
-            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "metric": METRICS[args.config], "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
             "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
             "dtype": "fp8e4m3+bf16", "data": "synthetic",
@@ -584,23 +737,25 @@ def run_reference(args):
     cfg = W.CONFIGS[args.config]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     wl = W.make_prefill(args.config, device=dev)
-    n_rows = max(4, oracle_threads())
+    n_rows = max(8, oracle_threads())
     for i in range(args.warmup):
-        oracle_sample(wl, max(1, n_rows // 4), seed=1000 + i)
-    secs = []
+        oracle_sample(wl, max(4, n_rows // 4), seed=1000 + i)
+    secs, vals = [], []
     for i in range(args.steps):
-        dt, desc = oracle_sample(wl, n_rows, seed=i)
+        dt, v, desc = oracle_sample(wl, n_rows, seed=i)
         secs.append(dt)
+        vals.append(v)
     step_s = float(np.mean(secs))
-    value = n_rows / step_s
+    value = float(np.mean(vals))
     line = {
-        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+        "impl": "reference", "metric": METRICS[args.config], "value": round(value, 4), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(step_s * 1e3, 1), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": f"{cfg.name} (one causal prefill)", "L": cfg.L, "k": cfg.k,
                    "H": cfg.H, "H_I": cfg.H_I, "d_I": cfg.d_I,
-                   "step": f"{n_rows} sampled query rows per step"},
+                   "step": f"{n_rows} stratified query rows per step; value extrapolated to "
+                           f"the whole workload by the per-row flop model"},
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": oracle_threads(),
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,

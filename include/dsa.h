@@ -323,6 +323,22 @@ DSA_API const char* dsa_status_string(dsa_status_t status);
  * (DSA_ERR_BOUNDS).  Returns DSA_OK if it was clear. */
 DSA_API dsa_status_t dsa_get_device_error(void* stream);
 
+/*
+ * Test hook for the failure detection of the kernels (not for production
+ * use; the pages have no counterpart).  Every wait inside a kernel is bounded:
+ * a wait that runs out records DSA_ERR_TIMEOUT in the device error word and
+ * the kernel winds down and returns, leaving the CUDA context usable.  This
+ * call lets a test exercise that path without faulting anything:
+ *  - wait_limit_ns: the longest a single wait may take in launches made
+ *    after this call (0 restores the default of 2 s);
+ *  - drop_first_key_load != 0: the NEXT dsa_indexer_logits launch (only that
+ *    one) leaves out the first key-tile load of every CTA, so the MMA
+ *    issuer's wait for that tile runs out; that launch's scores are then
+ *    incomplete and dsa_get_device_error() returns DSA_ERR_TIMEOUT.
+ * Process-wide host state, not thread-safe against concurrent launches.
+ */
+DSA_API void dsa_debug_fault_injection(uint64_t wait_limit_ns, int drop_first_key_load);
+
 /* Library version, "major.minor.patch". */
 DSA_API const char* dsa_version(void);
 

@@ -104,6 +104,13 @@ def _rows(rows, n_q):
     return _c(rows, np.int64)
 
 
+def _check(rc: int, name: str) -> None:
+    if rc == -2:
+        raise ValueError(f"{name}: an e4m3 input holds a NaN code (0x7F or 0xFF)")
+    if rc != 0:
+        raise ValueError(f"{name}: bad arguments")
+
+
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
 
@@ -132,8 +139,7 @@ def indexer(q8, q_scale, w, k8, k_scale, rows=None) -> np.ndarray:
     rc = _load().oracle_indexer(_ptr(q8), _ptr(_c(q_scale, np.float32)), _ptr(_c(w, np.float32)),
                                 _ptr(k8), _ptr(_c(k_scale, np.float32)), n_q, n_k, H_I, d_I,
                                 _ptr(rows), len(rows), _ptr(out), n_k)
-    if rc != 0:
-        raise ValueError("oracle_indexer: bad arguments")
+    _check(rc, "oracle_indexer")
     return out
 
 
@@ -193,8 +199,7 @@ def forward(q8, q_scale, w, k8, k_scale, q_bits, kv_bits, k, scale, d_v=512, row
                                 _ptr(k8), _ptr(_c(k_scale, np.float32)), _ptr(q_bits),
                                 _ptr(kv_bits), n_q, n_k, H_I, d_I, H, d_qk, d_v, k, float(scale),
                                 _ptr(rows), R, _ptr(idx), _ptr(out), _ptr(lse))
-    if rc != 0:
-        raise ValueError("oracle_forward: bad arguments")
+    _check(rc, "oracle_forward")
     return idx, out, lse
 
 
@@ -217,8 +222,7 @@ def forward_at(q8, q_scale, w, k8, k_scale, q_bits, kv_bits, pos, k, scale, d_v=
                                    _ptr(k8), _ptr(_c(k_scale, np.float32)), _ptr(q_bits),
                                    _ptr(kv_bits), _ptr(pos), R, n_k, H_I, d_I, H, d_qk, d_v, k,
                                    float(scale), _ptr(idx), _ptr(out), _ptr(lse))
-    if rc != 0:
-        raise ValueError("oracle_forward_at: bad arguments")
+    _check(rc, "oracle_forward_at")
     return idx, out, lse
 
 
@@ -235,8 +239,7 @@ def indexer_at(q8, q_scale, w, k8, k_scale, pos):
     rc = _load().oracle_indexer_at(_ptr(q8), _ptr(_c(q_scale, np.float32)), _ptr(_c(w, np.float32)),
                                    _ptr(k8), _ptr(_c(k_scale, np.float32)), _ptr(pos), R, n_k, H_I,
                                    d_I, _ptr(out), n_k)
-    if rc != 0:
-        raise ValueError("oracle_indexer_at: bad arguments")
+    _check(rc, "oracle_indexer_at")
     return out
 
 

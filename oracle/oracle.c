@@ -9,7 +9,8 @@
  *
  * Everything is computed in double precision straight from the definitions,
  * one query row at a time, with no blocking, fusion or reordering.  OpenMP
- * only spreads independent query rows over host cores.
+ * only spreads independent work over host cores: query rows, or the scores
+ * of one row (oracle_indexer_at).
  *
  * Sources (the pages this follows):
  *  - "DeepSeek V3.2 and the lightning indexer" (montana-research blog),
@@ -71,6 +72,15 @@ double oracle_e4m3_decode(uint8_t b) {
   return sign ? -v : v;
 }
 
+/* The e4m3 NaN codes (0x7F, 0xFF) are not values: an input that holds one is
+ * an error of the caller, reported instead of scored.  Returns 1 if any of
+ * the n bytes is such a code. */
+static int has_e4m3_nan(const uint8_t* b, int64_t n) {
+  for (int64_t i = 0; i < n; ++i)
+    if ((b[i] & 0x7F) == 0x7F) return 1;
+  return 0;
+}
+
 /* bfloat16 is the top half of an IEEE binary32. */
 double oracle_bf16_decode(uint16_t h) {
   uint32_t u = ((uint32_t)h) << 16;
@@ -110,6 +120,7 @@ int oracle_indexer(const uint8_t* q8, const float* q_scale, const float* w, cons
                    const float* k_scale, int64_t n_q, int64_t n_k, int H_I, int d_I,
                    const int64_t* rows, int64_t n_rows, double* out, int64_t ld_out) {
   if (n_q < 0 || n_k < n_q || H_I <= 0 || d_I <= 0 || ld_out < n_k) return -1;
+  if (has_e4m3_nan(q8, n_q * H_I * d_I) || has_e4m3_nan(k8, n_k * d_I)) return -2;
   int bad = 0;
 #pragma omp parallel for schedule(dynamic, 1)
   for (int64_t r = 0; r < n_rows; ++r) {
@@ -280,6 +291,7 @@ int oracle_forward(const uint8_t* q8, const float* q_scale, const float* w, cons
                    const int64_t* rows, int64_t n_rows, int32_t* idx_out, double* out,
                    double* lse) {
   if (k <= 0 || n_k < n_q || d_v > d_qk || H <= 0 || H_I <= 0 || d_I <= 0) return -1;
+  if (has_e4m3_nan(q8, n_q * H_I * d_I) || has_e4m3_nan(k8, n_k * d_I)) return -2;
   int bad = 0;
 #pragma omp parallel
   {
@@ -324,6 +336,7 @@ int oracle_forward_at(const uint8_t* q8, const float* q_scale, const float* w, c
                       int d_qk, int d_v, int k, double scale, int32_t* idx_out, double* out,
                       double* lse) {
   if (k <= 0 || d_v > d_qk || H <= 0 || H_I <= 0 || d_I <= 0 || !pos) return -1;
+  if (has_e4m3_nan(q8, n_rows * H_I * d_I) || has_e4m3_nan(k8, n_k * d_I)) return -2;
   int bad = 0;
 #pragma omp parallel
   {
@@ -363,18 +376,19 @@ int oracle_indexer_at(const uint8_t* q8, const float* q_scale, const float* w, c
                       const float* k_scale, const int64_t* pos, int64_t n_rows, int64_t n_k,
                       int H_I, int d_I, double* out, int64_t ld_out) {
   if (H_I <= 0 || d_I <= 0 || ld_out < n_k || !pos) return -1;
-  int bad = 0;
-#pragma omp parallel for schedule(dynamic, 1)
+  if (has_e4m3_nan(q8, n_rows * H_I * d_I) || has_e4m3_nan(k8, n_k * d_I)) return -2;
+  for (int64_t r = 0; r < n_rows; ++r)
+    if (pos[r] < 0 || pos[r] >= n_k) return -1;
+  /* Few, long rows are the use of this entry (sampled rows of a long
+   * sequence, decode rows), so the independent scores of a row are spread
+   * over the host cores rather than the rows. */
   for (int64_t r = 0; r < n_rows; ++r) {
-    int64_t p = pos[r];
-    if (p < 0 || p >= n_k) {
-      bad = 1;
-      continue;
-    }
+    const int64_t p = pos[r];
+#pragma omp parallel for schedule(static)
     for (int64_t s = 0; s <= p; ++s)
       out[r * ld_out + s] = indexer_score(q8, q_scale, w, k8, k_scale, r, s, H_I, d_I);
   }
-  return bad ? -1 : 0;
+  return 0;
 }
 
 /* Sparse attention of query rows given with their positions (row r of q at

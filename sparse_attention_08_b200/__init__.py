@@ -17,7 +17,7 @@ __all__ = [
     "dsa_forward_workspace_size", "dsa_get_device_error", "dsa_forward_noalloc",
     "dsa_forward_host", "dsa_forward_host_workspace_size", "dsa_indexer_kl",
     "dsa_indexer_kl_workspace_size", "dsa_masked_mha_fwd", "dsa_masked_mha_workspace_size",
-    "EXPORTED",
+    "dsa_debug_fault_injection", "EXPORTED",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -30,7 +30,7 @@ EXPORTED = (
     "dsa_forward_workspace_size", "dsa_status_string", "dsa_get_device_error", "dsa_version",
     "dsa_forward_noalloc", "dsa_forward_host", "dsa_forward_host_workspace_size",
     "dsa_indexer_kl", "dsa_indexer_kl_workspace_size", "dsa_masked_mha_fwd",
-    "dsa_masked_mha_workspace_size",
+    "dsa_masked_mha_workspace_size", "dsa_debug_fault_injection",
 )
 
 STATUS = {
@@ -90,10 +90,19 @@ def load():
     lib.dsa_status_string.restype = ctypes.c_char_p
     lib.dsa_get_device_error.argtypes = [P]
     lib.dsa_get_device_error.restype = I
+    lib.dsa_debug_fault_injection.argtypes = [ctypes.c_uint64, I]
+    lib.dsa_debug_fault_injection.restype = None
     lib.dsa_version.argtypes = []
     lib.dsa_version.restype = ctypes.c_char_p
     _lib = lib
     return lib
+
+
+def dsa_debug_fault_injection(wait_limit_ns: int = 0, drop_first_key_load: bool = False):
+    """Test hook: the wait limit of later launches (0 = the default 2 s) and a
+    one-shot request that the next dsa_indexer_logits launch leave out its
+    first key-tile load, so a bounded wait runs out (DSA_ERR_TIMEOUT)."""
+    load().dsa_debug_fault_injection(int(wait_limit_ns), 1 if drop_first_key_load else 0)
 
 
 def dsa_version() -> str:

@@ -22,6 +22,11 @@ __device__ unsigned g_dsa_err[2];  // [0] sticky error bits, [1] newest failed l
 
 std::atomic<unsigned> g_generation{1};
 
+// Test hook state (dsa_debug_fault_injection): the wait limit of later
+// launches (0 = the default) and a one-shot request for the indexer.
+std::atomic<uint64_t> g_wait_limit_ns{0};
+std::atomic<unsigned> g_inject_indexer{0};
+
 constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool ready = false;
@@ -63,6 +68,9 @@ dsa::DevErr next_err(const DeviceInfo* d) {
   dsa::DevErr e;
   e.word = d->err;
   e.gen = g_generation.fetch_add(1);
+  e.inject = 0;
+  const uint64_t lim = g_wait_limit_ns.load();
+  e.limit_ns = lim != 0 ? lim : dsa::kWaitLimitNs;
   return e;
 }
 
@@ -181,7 +189,9 @@ dsa_status_t dsa_indexer_logits(const void* q_fp8, const float* q_scale, const f
   a.logits = logits;
   a.ld = ld_logits;
   a.tile_n = tile_n;
-  return from_cuda(dsa::launch_indexer(tq, tk, a, dev->num_sms, next_err(dev),
+  dsa::DevErr err = next_err(dev);
+  err.inject = g_inject_indexer.exchange(0);
+  return from_cuda(dsa::launch_indexer(tq, tk, a, dev->num_sms, err,
                                        static_cast<cudaStream_t>(stream)));
 }
 
@@ -403,6 +413,11 @@ dsa_status_t dsa_forward(const void* q_fp8, const float* q_scale, const float* w
   if (st != DSA_OK) return st;
   return dsa_sparse_mla_fwd(q, kv, idx, cu_seqlens_q, cu_seqlens_k, B, max_len_q, max_len_k,
                             total_q, total_k, H, d_qk, d_v, k, sm_scale, out, lse, stream);
+}
+
+void dsa_debug_fault_injection(uint64_t wait_limit_ns, int drop_first_key_load) {
+  g_wait_limit_ns.store(wait_limit_ns);
+  g_inject_indexer.store(drop_first_key_load ? dsa::kInjectDropFirstKeyLoad : 0u);
 }
 
 dsa_status_t dsa_get_device_error(void* stream) {

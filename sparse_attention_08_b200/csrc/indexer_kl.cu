@@ -334,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_target_kernel(const Params P
     }
     mma_commit_warp(bar(kBDrain));
     if (lane == 0) {
-      mbar_wait_drain(bar(kBDrain), 0);
+      mbar_wait_drain(bar(kBDrain), 0, P.err);
       if (!ok) *abort_flag = 1;
     }
     __syncwarp();

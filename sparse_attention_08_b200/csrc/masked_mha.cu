@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) ok = issue_pv(n_tiles - 1);
     mma_commit_warp(drain);
-    if (lane == 0) mbar_wait_drain(drain, 0);
+    if (lane == 0) mbar_wait_drain(drain, 0, P.err);
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax

@@ -1,5 +1,5 @@
 // ptx.cuh -- hand-written inline-PTX wrappers for sm_100a used by the DSA
-// kernels: mbarriers with bounded waits, TMA tile and gather4 loads,
+// kernels: mbarriers with bounded waits, TMA tile loads, cp.async copies,
 // tcgen05 (TMEM allocation, MMA, commit, loads/stores) and the shared-memory
 // matrix / instruction descriptors.  Written from the PTX ISA description of
 // these instructions; bit layouts of the descriptors are spelled out below.
@@ -25,8 +25,17 @@ enum : unsigned {
 };
 
 struct DevErr {
-  unsigned* word;  // device address of unsigned[2]
-  unsigned gen;    // this launch's generation
+  unsigned* word;     // device address of unsigned[2]
+  unsigned gen;       // this launch's generation
+  unsigned inject;    // test hook, normally 0 (kInject* bits below)
+  uint64_t limit_ns;  // longest a single wait may take
+};
+
+// Test hooks carried by a launch (set only through dsa_debug_fault_injection):
+// the indexer's producer leaves out its first key-tile load, so the MMA
+// issuer's wait on it runs out and the launch ends with a timeout error.
+enum : unsigned {
+  kInjectDropFirstKeyLoad = 1u,
 };
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
@@ -44,7 +53,8 @@ __device__ __forceinline__ bool launch_failed(const DevErr& e) {
   return *reinterpret_cast<volatile unsigned*>(e.word + 1) >= e.gen;
 }
 
-// Longest a single wait may take before the kernel declares a timeout.
+// Longest a single wait may take before the kernel declares a timeout,
+// unless a test sets a shorter limit for its launches.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 // ---------------------------------------------------------------------------
@@ -84,8 +94,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Returns false (and
-// records a timeout) if it does not within kWaitLimitNs, or if another CTA of
-// the same launch has already failed.
+// records a timeout) if it does not within the launch's limit, or if another
+// CTA of the same launch has already failed.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const DevErr& e) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -93,7 +103,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const D
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (launch_failed(e)) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > e.limit_ns) {
         raise_error(e, kErrTimeout);
         return false;
       }
@@ -104,10 +114,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const D
 // Waits for a phase only by the clock (never gives up because of another
 // CTA): used on the way out after a failure, to let this CTA's own copies and
 // MMAs in flight land before its shared and tensor memory are released.
-__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, const DevErr& e) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (globaltimer_ns() - t0 > e.limit_ns) return false;
   }
   return true;
 }

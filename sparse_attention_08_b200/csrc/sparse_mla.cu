@@ -411,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t drain = drain_bar(warp == kMmaWarp ? 0 : 1);
     mma_commit_warp(drain);
     if (lane == 0) {
-      mbar_wait_drain(drain, 0);
+      mbar_wait_drain(drain, 0, P.err);
       if (!ok) *abort_flag = 1;
     }
     __syncwarp();

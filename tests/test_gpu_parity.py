@@ -171,8 +171,8 @@ def _attention_vs_oracle(cpu, gpu, idx_gpu):
                              np.concatenate(gl_all), np.concatenate(ol_all))
 
 
-# H <= 64 runs one CTA per 64-head group; H > 64 runs CTA pairs over
-# 128-head groups (192: a second group with only 64 real heads).
+# Every work item is (query, group of 64 heads): H = 16 and 32 fill part of
+# one group, 128 is two groups, 192 three and 256 four.
 @pytest.mark.parametrize("H,k", [(16, 64), (128, 100), (64, 256), (32, 130), (192, 128),
                                  (256, 64)])
 def test_attention_small(H, k):
@@ -413,19 +413,91 @@ def test_config2_sampled_bench_launch():
     assert torch.isfinite(out.float()).all()
 
 
-def test_config3_decode_sampled():
+def _attention_compact(q_rows_bits, kv_of_row, g_idx, pos, scale):
+    """Oracle attention of rows from different sequences in one call: row r's
+    valid selected latents (0 <= s <= pos[r]) are copied, in its index-row
+    order, into a compact latent array at rows r*k + j, and its index row is
+    renumbered to point there.  The oracle then sums exactly the same latents
+    in the same order (a relabelling of rows, no arithmetic)."""
+    R, k = g_idx.shape
+    d = q_rows_bits.shape[2]
+    kvc = np.zeros((R * k, d), dtype=np.uint16)
+    idxc = np.full((R, k), -1, dtype=np.int32)
+    for r in range(R):
+        valid = (g_idx[r] >= 0) & (g_idx[r] <= pos[r])
+        j = np.flatnonzero(valid)
+        kvc[r * k + j] = kv_of_row(r, g_idx[r, j])
+        idxc[r, j] = r * k + j
+    pos_c = np.array([r * k + k - 1 for r in range(R)], dtype=np.int64)
+    return oracle.sparse_mla_at(q_rows_bits, kvc, idxc, pos_c, scale)
+
+
+def test_config3_decode_all_rows():
+    # every one of the 64 decode rows (ragged caches of 4K..131K keys), in the
+    # launch configuration the bench times
     wl = W.make_decode(3, device="cuda")
     idx, out, lse = C.gpu_forward(wl)
     C.assert_no_device_error()
-    for b in (0, 17, 63):
-        _sampled_parity(wl, b, np.array([0]), idx, out, lse)
+    g_idx = C.np_(idx)
+    q8, qs, w = C.np_(wl.q8), C.np_(wl.q_scale), C.np_(wl.w)
+    k8_all, ks_all = C.np_(wl.k8), C.np_(wl.k_scale)
+    cu_k = C.np_(wl.cu_k).astype(np.int64)
+    pos = []
+    for b in range(wl.B):
+        k0, k1 = int(cu_k[b]), int(cu_k[b + 1])
+        p = k1 - k0 - 1
+        pos.append(p)
+        sc = oracle.indexer_at(q8[b:b + 1], qs[b:b + 1], w[b:b + 1], k8_all[k0:k1],
+                               ks_all[k0:k1], np.array([p]))
+        o_idx = oracle.topk(sc, 1, wl.k)
+        C.check_topk_near_cut(g_idx[b:b + 1], o_idx, sc, [p], wl.k)
+
+    def kv_of_row(r, s):
+        rows = torch.as_tensor(cu_k[r] + s, device="cuda")
+        return C.bits(wl.kv[rows])
+
+    o, ol = _attention_compact(C.bits(wl.q), kv_of_row, g_idx, np.array(pos), wl.scale)
+    C.check_attention(C.np_(out.float()), o, C.np_(lse), ol)
 
 
-def test_config4_last_chunk_sampled():
+def test_config4_every_chunk_sampled():
+    # the 131072-token prefill as 8 chunks of 16384 queries against the
+    # growing cache, each chunk through dsa_forward as the bench runs it;
+    # sampled rows of every chunk (its first and last query and one drawn
+    # row, plus positions k-2..k+1 in chunk 0) go to the oracle together
     full = W.make_prefill(4, device="cuda")
-    C_ = full.cfg.L // full.cfg.chunks
-    wl = W.chunk_of(full, full.cfg.chunks - 1, C_)
-    idx, out, lse = C.gpu_forward(wl)
-    C.assert_no_device_error()
-    rows = _sample_rows(wl.T_q, wl.T_k, wl.k, 3, seed=4)
-    _sampled_parity(wl, 0, rows, idx, out, lse)
+    n_ch = full.cfg.chunks
+    C_ = full.cfg.L // n_ch
+    rng = np.random.default_rng(4)
+    rows, g_idx, g_out, g_lse = [], [], [], []
+    for c in range(n_ch):
+        wl = W.chunk_of(full, c, C_)
+        idx, out, lse = C.gpu_forward(wl)
+        C.assert_no_device_error()
+        # properties that hold at any size, on every row of the chunk
+        g = C.np_(idx)
+        p_all = np.arange(c * C_, (c + 1) * C_)
+        assert np.array_equal((g >= 0).sum(axis=1), np.minimum(p_all + 1, wl.k))
+        assert np.all(np.diff(g, axis=1)[(g >= 0)[:, 1:]] > 0)
+        assert torch.isfinite(out.float()).all()
+        loc = {0, C_ - 1, int(rng.integers(1, C_ - 1))}
+        if c == 0:
+            loc |= {wl.k - 2, wl.k - 1, wl.k, wl.k + 1}
+        loc = np.array(sorted(loc), dtype=np.int64)
+        t = torch.as_tensor(loc, device="cuda")
+        rows.append(c * C_ + loc)
+        g_idx.append(g[loc])
+        g_out.append(C.np_(out[t].float()))
+        g_lse.append(C.np_(lse[t]))
+        del idx, out, lse, wl
+        torch.cuda.empty_cache()
+    rows = np.concatenate(rows)
+    g_idx, g_out, g_lse = np.concatenate(g_idx), np.concatenate(g_out), np.concatenate(g_lse)
+    t = torch.as_tensor(rows, device="cuda")
+    sc = oracle.indexer_at(C.np_(full.q8[t]), C.np_(full.q_scale[t]), C.np_(full.w[t]),
+                           C.np_(full.k8), C.np_(full.k_scale), rows)
+    o_idx = np.stack([oracle.topk(sc[r:r + 1, : p + 1], 1, full.k)[0]
+                      for r, p in enumerate(rows)])
+    C.check_topk_near_cut(g_idx, o_idx, sc, list(rows), full.k)
+    o, ol = oracle.sparse_mla_at(C.bits(full.q[t]), C.bits(full.kv), g_idx, rows, full.scale)
+    C.check_attention(g_out, o, g_lse, ol)

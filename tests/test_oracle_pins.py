@@ -61,6 +61,31 @@ def test_e4m3_decode_matches_torch_all_codes():
     assert oracle.e4m3_decode(0xB8) == -1.0
 
 
+@pytest.mark.parametrize("where", ["q", "k"])
+@pytest.mark.parametrize("code", [0x7F, 0xFF])
+def test_indexer_refuses_e4m3_nan_codes(where, code):
+    # 0x7F / 0xFF are the format's NaN encodings, not values: every oracle
+    # entry that decodes e4m3 reports them as an input error
+    wl = W.make_small(H_I=4, d_I=64, H=16, L=40, k=8, integer=True, seed=3)
+    q8, k8 = _np(wl.q8).copy(), _np(wl.k8).copy()
+    if where == "q":
+        q8[7, 2, 5] = code
+    else:
+        k8[3, 11] = code
+    qs, w, ks = _np(wl.q_scale), _np(wl.w), _np(wl.k_scale)
+    pos = np.array([39], dtype=np.int64)
+    with pytest.raises(ValueError, match="NaN code"):
+        oracle.indexer(q8, qs, w, k8, ks)
+    with pytest.raises(ValueError, match="NaN code"):
+        oracle.indexer_at(q8[-1:] if where == "k" else q8[7:8], qs[:1], w[:1], k8, ks, pos)
+    qb, kvb = _bits(wl.q), _bits(wl.kv)
+    with pytest.raises(ValueError, match="NaN code"):
+        oracle.forward(q8, qs, w, k8, ks, qb, kvb, wl.k, wl.scale)
+    with pytest.raises(ValueError, match="NaN code"):
+        oracle.forward_at(q8[7:8], qs[:1], w[:1], k8, ks, qb[:1], kvb, np.array([39]), wl.k,
+                          wl.scale)
+
+
 def test_bf16_decode_matches_torch():
     g = torch.Generator().manual_seed(1)
     x = (torch.randn(4096, generator=g) * 100).to(torch.bfloat16)
