@@ -227,44 +227,52 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int64_t qc = 0, kc = 0, ac = 0;
-      bool ok = true;
-      for (int64_t item = blockIdx.x; ok && item < P.n_items; item += gridDim.x) {
-        Item it;
-        if (!decode_item<QPT>(item, P, it)) continue;
-        const int qb = static_cast<int>(qc & 1);
-        if (!(ok = mbar_wait(q_full(qb), static_cast<uint32_t>((qc >> 1) & 1), P.err))) break;
-        const uint32_t q_addr = sbase + L::kOffQ + qb * L::kQBytes;
-        for (int j = 0; j < it.nkb; ++j) {
-          const int st = static_cast<int>(kc % kStages);
-          if (!(ok = mbar_wait(k_full(st), static_cast<uint32_t>((kc / kStages) & 1), P.err))) break;
-          const int ab = static_cast<int>(ac % kBufs);
-          if (!(ok = mbar_wait(acc_empty(ab), static_cast<uint32_t>(((ac / kBufs) & 1) ^ 1), P.err)))
-            break;
-          tc_fence_after();
-          const uint32_t k_addr = sbase + L::kOffK + st * L::kKBytes;
-          const uint32_t d = tmem + static_cast<uint32_t>(ab) * kN;
+    // The whole warp walks the items in lockstep and one elected lane issues
+    // a tile's MMAs; every operand is warp-uniform and the descriptors are
+    // built once: a stage or query buffer adds a multiple of its size (in
+    // 16-byte units) to the start-address field.
+    int64_t qc = 0, kc = 0, ac = 0;
+    bool ok = true;
+    const uint64_t a0 = smem_desc(sbase + L::kOffK, 16, L::kSbo, L::kSwizzle);
+    const uint64_t b0 = smem_desc(sbase + L::kOffQ, 16, L::kSbo, L::kSwizzle);
+    for (int64_t item = blockIdx.x; ok && item < P.n_items; item += gridDim.x) {
+      Item it;
+      if (!decode_item<QPT>(item, P, it)) continue;
+      const int qb = static_cast<int>(qc & 1);
+      if (!(ok = warp_wait(q_full(qb), static_cast<uint32_t>((qc >> 1) & 1), P.err))) break;
+      const uint64_t bq = b0 + ((static_cast<uint32_t>(qb) * L::kQBytes) >> 4);
+      for (int j = 0; j < it.nkb; ++j) {
+        const int st = static_cast<int>(kc % kStages);
+        const int ab = static_cast<int>(ac % kBufs);
+        ok = warp_wait(k_full(st), static_cast<uint32_t>((kc / kStages) & 1), P.err) &&
+             warp_wait(acc_empty(ab), static_cast<uint32_t>(((ac / kBufs) & 1) ^ 1), P.err);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t ak = a0 + ((static_cast<uint32_t>(st) * L::kKBytes) >> 4);
+        const uint32_t d = tmem + static_cast<uint32_t>(ab) * kN;
+        if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < D_I / 32; ++kk) {
-            const uint64_t adesc = smem_desc(k_addr + kk * 32, 16, L::kSbo, L::kSwizzle);
-            const uint64_t bdesc = smem_desc(q_addr + kk * 32, 16, L::kSbo, L::kSwizzle);
-            mma_f8(d, adesc, bdesc, L::kIdesc, kk > 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < D_I / 32; ++kk)
+            mma_f8(d, ak + (kk * 32 >> 4), bq + (kk * 32 >> 4), L::kIdesc, kk > 0 ? 1u : 0u);
           mma_commit(k_empty(st));
           mma_commit(acc_full(ab));
-          ++kc;
-          ++ac;
         }
-        if (!ok) break;
-        mma_commit(q_empty(qb));
-        ++qc;
+        __syncwarp();
+        ++kc;
+        ++ac;
       }
-      // every MMA issued by this thread completes before TMEM is released
-      mma_commit(drain_bar);
+      if (!ok) break;
+      if (elect_one()) mma_commit(q_empty(qb));
+      __syncwarp();
+      ++qc;
+    }
+    // every MMA issued by this warp completes before TMEM is released
+    mma_commit_warp(drain_bar);
+    if (lane == 0) {
       mbar_wait_drain(drain_bar, 0, P.err);
       if (!ok) *abort_flag = 1;
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     // Warpgroup eg reads accumulator buffer eg / kHalves (every kBufs-th
@@ -307,6 +315,10 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
       for (int j = 0; j < it.nkb; ++j, ++ac) {
         const int ab = static_cast<int>(ac % kBufs);
         if (ab != ab_mine) continue;
+        // the key's scale is fetched before the accumulator is waited for,
+        // so its latency hides behind the MMA
+        const int s_local = (it.kb0 + j) * kBlockK + row;
+        const float ks = s_local < it.len_k ? __ldg(P.k_scale + it.k_row0 + s_local) : 0.f;
         // each warp waits and releases on its own: no warpgroup barrier per tile
         if (!warp_wait(acc_full(ab), static_cast<uint32_t>((ac / kBufs) & 1), P.err)) {
           *abort_flag = 1;
@@ -314,7 +326,6 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
           break;
         }
         tc_fence_after();
-        const int s_local = (it.kb0 + j) * kBlockK + row;
         float2 acc[QH][NCH];
 #pragma unroll
         for (int qi = 0; qi < QH; ++qi) {
@@ -323,8 +334,10 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
         }
         const uint32_t dcol = tmem + lane_addr + static_cast<uint32_t>(ab) * kN + hf * kHalf;
 #pragma unroll
+        // Columns of queries past the group's last one (a sequence's last
+        // group) carry weight 0 and add exactly nothing; their scores are not
+        // stored, so every tile is read out alike, without branches.
         for (int cg = 0; cg < kHalf / 32; cg += kChunksPerWait) {
-          if ((hf * kHalf + cg * 32) / H_I >= it.nq) break;
           uint32_t v[kChunksPerWait][32];
 #pragma unroll
           for (int u = 0; u < kChunksPerWait; ++u) tmem_ld_32x32b_x32(dcol + (cg + u) * 32, v[u]);
@@ -350,7 +363,6 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty(ab));
         if (s_local < it.len_k) {
-          const float ks = __ldg(P.k_scale + it.k_row0 + s_local);
           const int p0 = it.len_k - it.len_q + it.q0;
 #pragma unroll
           for (int ql = 0; ql < QH; ++ql) {

@@ -7,27 +7,43 @@
 // min(k, n) largest, ties to the lower position, -0.0 == +0.0, written in
 // ascending position order and padded with -1.
 //
-// How: one CTA of 256 threads (8 warps) per row, three CTAs per SM; scores
+// How: a row is handled by a cluster of C CTAs of 256 threads.  C = 1 when
+// the batch has enough rows to fill the GPU: a persistent grid of a few CTAs
+// per SM walks the rows and pulls each CTA's next row into L2 while it works
+// on the current one.  C = 8 for a few long rows (a decode batch).  Scores
 // map to order-preserving 32-bit keys (larger float -> larger unsigned key,
-// -0 folded into +0).  Warp w owns the w-th contiguous eighth of the row and
-// the w-th eighth of a shared candidate buffer, so candidates stay in
+// -0 folded into +0).  The row's 16-byte groups are cut into 8C contiguous
+// segments in position order; warp w of cluster rank c owns segment 8c + w
+// and the w-th region of its CTA's candidate buffer, so candidates stay in
 // position order without any sorting.
-//  1. Threshold estimate (rows longer than the candidate buffer).  1024
-//     evenly spaced samples give, by an exact radix select among them, a key
-//     t0 that with a wide safety margin lies below the row's k-th largest.
-//  2. Filter.  Each warp streams its segment once from memory (16-byte
-//     loads, eight in flight per lane) and appends every (position, key)
-//     with key >= t0 to its region, in position order (ballot + prefix).
-//  3. Exact select among the candidates: radix passes of 8 bits, starting
-//     below the bits that all candidates share, give the exact k-th key T
-//     and how many keys equal to T are kept (krem).
-//  4. Ordered output.  Warps walk their regions in order; a key is kept if
-//     it is > T or it is one of the first krem keys == T (tie ranks from a
-//     prefix over the regions); output slots come from a second prefix.
-// If the estimate fails (fewer than k candidates, or a region overflows,
-// e.g. rows of massive ties), the row falls back to exact radix passes over
-// the whole row in global memory followed by an ordered ballot-scan
-// compaction.  Both routes give the same, unique answer.
+//  1. Threshold.  Rows longer than about 2k (or than the candidate buffers)
+//     draw S evenly spaced samples (S = 1024, or 4096 past 32768 scores).
+//     Two levels of 2048-bin histograms of their keys (over [min, max], then
+//     inside the bin holding the r0-th largest sample) give a key t0, the
+//     lower edge of the fine bin holding that sample, with at least r0
+//     samples at or above it; r0 = E + 4 sqrt(E) + 8 for E = S k / n
+//     expected samples above the row's k-th largest, so t0 lies below that
+//     score with a wide margin.  Every CTA of a cluster computes the same t0.
+//  2. Filter.  Each warp streams its segment once (16-byte loads), compares
+//     the raw floats with t0 as a float, and appends the (key, position) of
+//     every score that passes to its region in position order (ballot
+//     prefix), tracking the candidates' key range.
+//  3. Exact k-th key.  Two levels of 2048-bin histograms of the candidates
+//     (over their key range, then inside the bin that holds the k-th largest;
+//     summed over the cluster through distributed shared memory) find a fine
+//     bin holding the k-th largest and how many keys lie above it; the few
+//     keys of that bin are gathered and ranked against each other, which
+//     gives the k-th key T and how many keys equal to T are kept (krem).
+//  4. Ordered output.  A key is kept if it is > T or one of the first krem
+//     keys == T in position order (tie ranks from prefixes over the cluster's
+//     CTAs and their warps); output slots come from a second prefix.
+// If the threshold fails (fewer than k candidates, or a region overflows,
+// e.g. rows of massive ties) or the cut bin holds too many keys, rank 0 falls
+// back to exact radix passes over the whole row in global memory and an
+// ordered ballot-scan compaction.  Both routes give the same, unique answer.
+// Every decision that changes how many cluster barriers a CTA passes is taken
+// from values that all CTAs of the cluster read alike.
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -38,12 +54,16 @@
 namespace dsa {
 namespace {
 
+namespace cg = cooperative_groups;
+
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kCap = 8192;                 // candidate buffer entries
-constexpr int kRegion = kCap / kWarps;     // per warp
-constexpr int kSamples = 1024;
 constexpr int kUnroll = 8;                 // 16-byte loads in flight per lane
+constexpr int kSplitC = 8;                 // CTAs per row for few long rows
+constexpr int kBins = 2048;                // histogram bins (11 bits)
+constexpr int kBinBits = 11;
+constexpr int kBinsPerThread = kBins / kThreads;
+constexpr int kList = 512;                 // keys of the cut bin ranked directly
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -51,23 +71,80 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The float whose key is u (inverse of order_key on the keys it produces):
+// x >= key_float(order_key(y)) exactly when order_key(x) >= order_key(y).
+__device__ __forceinline__ float key_float(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
+// Bin shift that maps keys in [lo, hi] onto at most kBins bins.
+__device__ __forceinline__ int bin_shift(uint32_t lo, uint32_t hi) {
+  const uint32_t span = hi - lo;
+  const int bits = span == 0u ? 0 : 32 - __clz(span);
+  return bits > kBinBits ? bits - kBinBits : 0;
+}
+
+// Values a CTA shares with the other CTAs of its cluster.
+enum { kXCand = 0, kXOverflow, kXMin, kXMax, kXList, kXGt, kXEq, kXCount };
+
+template <int CAP>
 struct Shared {
-  uint32_t hist[256];
+  uint32_t hist[kBins];
   uint32_t wsum[kWarps];
   uint32_t wsum2[kWarps];
   uint32_t wcnt[kWarps];       // candidates per region
   uint32_t red_min, red_max;
   uint32_t sel_digit;
   uint32_t cnt_above;
-  uint32_t overflow;
   uint32_t out_pos;
   uint32_t eq_seen;
-  uint32_t cand_key[kCap];
-  int32_t cand_pos[kCap];
+  uint32_t list_n;
+  uint32_t res_key, res_rem;
+  uint32_t xch[kXCount];
+  uint32_t xall[kSplitC][kXCount];   // every CTA's xch, gathered once (clusters)
+  uint32_t tot[kBins / kSplitC];     // cluster totals of the bins this CTA owns
+  uint32_t list_key[kList];
+  uint32_t mlist[kList];             // the cluster's cut-bin keys, gathered
+  uint32_t cand_key[CAP];
+  int32_t cand_pos[CAP];
 };
 
+// Cluster of C CTAs working on one row; with C == 1 a plain CTA.
+template <int C>
+struct Cluster {
+  __device__ __forceinline__ static unsigned rank() {
+    if constexpr (C == 1) return 0;
+    else return cg::this_cluster().block_rank();
+  }
+  __device__ __forceinline__ static void sync() {
+    if constexpr (C == 1) __syncthreads();
+    else cg::this_cluster().sync();
+  }
+  // Address of `p` (a location in this CTA's shared memory) in CTA r.
+  template <class T>
+  __device__ __forceinline__ static T* at(T* p, unsigned r) {
+    if constexpr (C == 1) return p;
+    else return cg::this_cluster().map_shared_rank(p, r);
+  }
+};
+
+// Copies every cluster CTA's xch into sh.xall (after a cluster barrier that
+// follows the writes), with independent remote loads.
+template <int C, int CAP>
+__device__ __forceinline__ void gather_xch(Shared<CAP>& sh) {
+  if constexpr (C > 1) {
+    if (threadIdx.x < C * kXCount) {
+      const unsigned q = threadIdx.x / kXCount, f = threadIdx.x % kXCount;
+      sh.xall[q][f] = Cluster<C>::at(sh.xch, q)[f];
+    }
+    __syncthreads();
+  }
+}
+
 // Block-wide exclusive scan of one value per thread; *total gets the sum.
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* buf, uint32_t* total) {
+template <int CAP>
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, Shared<CAP>& sh,
+                                                    uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t x = v;
 #pragma unroll
@@ -75,12 +152,12 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* buf, u
     const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
-  if (lane == 31) buf[warp] = x;
+  if (lane == 31) sh.wsum[warp] = x;
   __syncthreads();
   uint32_t before = 0, tot = 0;
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) {
-    const uint32_t s = buf[w];
+    const uint32_t s = sh.wsum[w];
     before += w < warp ? s : 0u;
     tot += s;
   }
@@ -89,20 +166,19 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* buf, u
   return before + x - v;
 }
 
-// Key source of a radix select: either the candidate regions in shared
-// memory (warp w scans region w) or a whole score row in global memory
-// (block-strided).
-struct RegionKeys {
-  const Shared* sh;
+// Key sources.  for_each(f) calls f(key) on every key.
+template <int CAP>
+struct RegionKeys {              // the candidate regions (warp w scans region w)
+  const Shared<CAP>* sh;
   template <class F>
   __device__ __forceinline__ void for_each(F f) const {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t cnt = sh->wcnt[warp];
-    const uint32_t* keys = sh->cand_key + warp * kRegion;
+    const uint32_t* keys = sh->cand_key + warp * (CAP / kWarps);
     for (uint32_t i = lane; i < cnt; i += 32) f(keys[i]);
   }
 };
-struct RowKeys {
+struct RowKeys {                 // a whole score row in global memory
   const float* row;
   int n;
   template <class F>
@@ -111,19 +187,28 @@ struct RowKeys {
   }
 };
 
-// Exact kk-th largest key (kk >= 1, at most the number of keys); krem
-// returns how many keys equal to it belong to the kk largest.  The bits that
-// all keys share are found first (block min / max); radix passes of 8 bits
-// then resolve the rest from the highest differing bit down.  All threads
-// return the same values.
+// The keys of `base` that fall into one bin of (key - lo) >> shift.
 template <class Keys>
-__device__ uint32_t select_kth(const Keys& keys, uint32_t kk, uint32_t& krem, Shared& sh) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t mn = 0xffffffffu, mx = 0u;
-  keys.for_each([&](uint32_t u) {
-    mn = min(mn, u);
-    mx = max(mx, u);
-  });
+struct BinKeys {
+  Keys base;
+  uint32_t lo;
+  int shift;
+  uint32_t bin;
+  template <class F>
+  __device__ __forceinline__ void for_each(F f) const {
+    const uint32_t l = lo, b = bin;
+    const int sh = shift;
+    base.for_each([&](uint32_t u) {
+      if (((u - l) >> sh) == b) f(u);
+    });
+  }
+};
+
+// The cluster-wide min and max of per-thread key ranges; every thread of
+// every CTA gets the same result in sh.red_min / sh.red_max.
+template <int CC, int CAP>
+__device__ void cluster_minmax(uint32_t mn, uint32_t mx, Shared<CAP>& sh) {
+  const int lane = threadIdx.x & 31;
   mn = __reduce_min_sync(0xffffffffu, mn);
   mx = __reduce_max_sync(0xffffffffu, mx);
   if (threadIdx.x == 0) {
@@ -136,22 +221,127 @@ __device__ uint32_t select_kth(const Keys& keys, uint32_t kk, uint32_t& krem, Sh
     atomicMax(&sh.red_max, mx);
   }
   __syncthreads();
+  if constexpr (CC > 1) {
+    if (threadIdx.x == 0) {
+      sh.xch[kXMin] = sh.red_min;
+      sh.xch[kXMax] = sh.red_max;
+    }
+    Cluster<CC>::sync();
+    gather_xch<CC>(sh);
+    if (threadIdx.x == 0) {
+      uint32_t a = 0xffffffffu, b = 0u;
+      for (unsigned r = 0; r < CC; ++r) {
+        a = min(a, sh.xall[r][kXMin]);
+        b = max(b, sh.xall[r][kXMax]);
+      }
+      sh.red_min = a;
+      sh.red_max = b;
+    }
+    Cluster<CC>::sync();   // every CTA has read xch before it is written again
+  }
+}
+
+// Histogram cut: bins of (key - lo) >> shift over the cluster's keys; finds
+// the bin holding the kk-th largest key (sh.sel_digit) and how many keys lie
+// in higher bins (sh.cnt_above).  kk >= 1 and at most the number of keys.
+template <int CC, int CAP, class Keys>
+__device__ void hist_cut(const Keys& keys, uint32_t kk, uint32_t lo, int shift, Shared<CAP>& sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int i = 0; i < kBinsPerThread; ++i) sh.hist[threadIdx.x + i * kThreads] = 0u;
+  __syncthreads();
+  keys.for_each([&](uint32_t u) { atomicAdd(&sh.hist[(u - lo) >> shift], 1u); });
+  // thread t owns bins kBins-1-8t .. kBins-8-8t, counted from the top down
+  uint32_t h[kBinsPerThread];
+  uint32_t s = 0;
+  if constexpr (CC > 1) {
+    // CTA q adds up bins q*kBins/CC .. (q+1)*kBins/CC - 1 over the cluster
+    // (thread t one bin, the CC remote loads issued together), then every
+    // CTA reads the totals it scans from their owners
+    static_assert(kBins / CC == kThreads, "one owned bin per thread");
+    Cluster<CC>::sync();                        // every CTA's histogram is complete
+    {
+      const unsigned me = Cluster<CC>::rank();
+      const int b = static_cast<int>(me) * kThreads + static_cast<int>(threadIdx.x);
+      uint32_t v[CC];
+#pragma unroll
+      for (int r = 0; r < CC; ++r) v[r] = Cluster<CC>::at(sh.hist, r)[b];
+      uint32_t t = 0;
+#pragma unroll
+      for (int r = 0; r < CC; ++r) t += v[r];
+      sh.tot[threadIdx.x] = t;
+    }
+    Cluster<CC>::sync();                        // every owner's totals are complete
+    {
+      const int b0 = kBins - 1 - kBinsPerThread * static_cast<int>(threadIdx.x);   // top bin
+      const unsigned owner = static_cast<unsigned>(b0) / kThreads;               // same for all 8
+      const uint32_t* tt = Cluster<CC>::at(sh.tot, owner);
+#pragma unroll
+      for (int i = 0; i < kBinsPerThread; ++i) h[i] = tt[(b0 - i) % kThreads];
+#pragma unroll
+      for (int i = 0; i < kBinsPerThread; ++i) s += h[i];
+    }
+  } else {
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kBinsPerThread; ++i) {
+      h[i] = sh.hist[kBins - 1 - kBinsPerThread * threadIdx.x - i];
+      s += h[i];
+    }
+  }
+  uint32_t x = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh.wsum[warp] = x;
+  __syncthreads();
+  uint32_t before = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) before += w < warp ? sh.wsum[w] : 0u;
+  uint32_t c = before + x - s;                  // keys in the bins above this thread's
+  if (c < kk && c + s >= kk) {
+#pragma unroll
+    for (int i = 0; i < kBinsPerThread; ++i) {
+      if (c < kk && c + h[i] >= kk) {
+        sh.sel_digit = static_cast<uint32_t>(kBins - 1 - kBinsPerThread * threadIdx.x - i);
+        sh.cnt_above = c;
+      }
+      c += h[i];
+    }
+  }
+  if constexpr (CC > 1) Cluster<CC>::sync();    // no CTA clears its histogram while read
+  else __syncthreads();
+}
+
+// Exact kk-th largest key by radix passes (kk >= 1, at most the number of
+// keys) over one CTA's keys; krem returns how many keys equal to it belong to
+// the kk largest.  Used on the fallback path only.
+template <int CAP, class Keys>
+__device__ uint32_t radix_select(const Keys& keys, uint32_t kk, uint32_t& krem, Shared<CAP>& sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t mn = 0xffffffffu, mx = 0u;
+  keys.for_each([&](uint32_t u) {
+    mn = min(mn, u);
+    mx = max(mx, u);
+  });
+  cluster_minmax<1>(mn, mx, sh);
   const uint32_t diff = sh.red_min ^ sh.red_max;
   krem = kk;
-  if (diff == 0u) return sh.red_max;               // every key is equal
-  const int top = 31 - __clz(diff);                 // highest differing bit
+  if (diff == 0u) return sh.red_max;              // every key is equal
+  const int top = 31 - __clz(diff);
   uint32_t mask = top == 31 ? 0u : ~((2u << top) - 1u);
   uint32_t prefix = sh.red_max & mask;
   for (int hi = top; hi >= 0; hi -= 8) {
     const int lo = hi >= 7 ? hi - 7 : 0;
     const uint32_t dmask = (2u << (hi - lo)) - 1u;
-    sh.hist[threadIdx.x] = 0u;                      // 256 threads, 256 bins
+    sh.hist[threadIdx.x] = 0u;
     __syncthreads();
     keys.for_each([&](uint32_t u) {
       if ((u & mask) == prefix) atomicAdd(&sh.hist[(u >> lo) & dmask], 1u);
     });
     __syncthreads();
-    // thread t owns bin 255 - t: an inclusive scan from the top bin down
     const uint32_t h = sh.hist[255 - threadIdx.x];
     uint32_t x = h;
 #pragma unroll
@@ -178,11 +368,12 @@ __device__ uint32_t select_kth(const Keys& keys, uint32_t kk, uint32_t& krem, Sh
 }
 
 // Fallback: exact select over the whole row in global memory, then an
-// ordered ballot-scan compaction.
+// ordered ballot-scan compaction (one CTA).
+template <int CAP>
 __device__ void topk_row_global(const float* __restrict__ row, int n, int k, int32_t* out,
-                                float* vout, Shared& sh) {
+                                float* vout, Shared<CAP>& sh) {
   uint32_t krem;
-  const uint32_t T = select_kth(RowKeys{row, n}, static_cast<uint32_t>(k), krem, sh);
+  const uint32_t T = radix_select(RowKeys{row, n}, static_cast<uint32_t>(k), krem, sh);
   if (threadIdx.x == 0) {
     sh.out_pos = 0;
     sh.eq_seen = 0;
@@ -198,9 +389,9 @@ __device__ void topk_row_global(const float* __restrict__ row, int n, int k, int
     const uint32_t eq_seen = sh.eq_seen;
     const uint32_t pos_base = sh.out_pos;
     uint32_t eq_tot, take_tot;
-    const uint32_t eq_rank = block_excl_scan(eq ? 1u : 0u, sh.wsum, &eq_tot);
+    const uint32_t eq_rank = block_excl_scan(eq ? 1u : 0u, sh, &eq_tot);
     const bool take = gt || (eq && eq_seen + eq_rank < krem);
-    const uint32_t pos = block_excl_scan(take ? 1u : 0u, sh.wsum, &take_tot);
+    const uint32_t pos = block_excl_scan(take ? 1u : 0u, sh, &take_tot);
     if (take) {
       out[pos_base + pos] = j;
       if (vout) vout[pos_base + pos] = f;
@@ -213,11 +404,13 @@ __device__ void topk_row_global(const float* __restrict__ row, int n, int k, int
   }
 }
 
-// Appends, in lane order, the flagged keys of this lane (flags bit e for
-// key[e], position pos0 + e) to the warp's region; returns the new count.
+// Appends, in lane order, the flagged entries of this lane (flags bit e for
+// v[e], position pos0 + e) to the warp's region and widens the lane's key
+// range; returns the new count.
+template <int CAP>
 __device__ __forceinline__ uint32_t region_append(uint32_t* rk, int32_t* rp, uint32_t cnt,
-                                                  const uint32_t (&key)[4], uint32_t flags,
-                                                  int pos0) {
+                                                  const float (&v)[4], uint32_t flags, int pos0,
+                                                  uint32_t& mn, uint32_t& mx) {
   const int lane = threadIdx.x & 31;
   const uint32_t c = __popc(flags);
   const uint32_t lt = (1u << lane) - 1u;
@@ -228,8 +421,11 @@ __device__ __forceinline__ uint32_t region_append(uint32_t* rk, int32_t* rp, uin
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     if ((flags >> e) & 1u) {
-      if (pos < kRegion) {
-        rk[pos] = key[e];
+      const uint32_t u = order_key(v[e]);
+      mn = min(mn, u);
+      mx = max(mx, u);
+      if (pos < static_cast<uint32_t>(CAP / kWarps)) {
+        rk[pos] = u;
         rp[pos] = pos0 + e;
       }
       ++pos;
@@ -238,64 +434,76 @@ __device__ __forceinline__ uint32_t region_append(uint32_t* rk, int32_t* rp, uin
   return cnt + __popc(b0) + 2u * __popc(b1) + 4u * __popc(b2);
 }
 
-__global__ void __launch_bounds__(kThreads, 3)
-    topk_kernel(const float* __restrict__ logits, int64_t ld, const int32_t* __restrict__ cu_q,
-                const int32_t* __restrict__ cu_k, int B, int k, int32_t* __restrict__ idx,
-                float* __restrict__ val) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  Shared& sh = *reinterpret_cast<Shared*>(smem_raw);
+// One row: the whole pipeline, by every thread of every CTA of the cluster.
+template <int C, int CAP>
+__device__ void topk_row(const float* __restrict__ row, int n, int k, int32_t* __restrict__ out,
+                         float* __restrict__ vout, Shared<CAP>& sh) {
+  constexpr int kRegion = CAP / kWarps;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned crank = Cluster<C>::rank();
 
-  const int64_t r = blockIdx.x;
-  int lo = 0, hi = B;  // cu_q[lo] <= r < cu_q[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(cu_q + mid) <= r) lo = mid; else hi = mid;
-  }
-  const int b = lo;
-  const int len_q = __ldg(cu_q + b + 1) - __ldg(cu_q + b);
-  const int len_k = __ldg(cu_k + b + 1) - __ldg(cu_k + b);
-  const int i = static_cast<int>(r - __ldg(cu_q + b));
-  const int n = len_k - len_q + i + 1;  // candidates 0..p
-  const float* row = logits + r * ld;
-  int32_t* out = idx + r * k;
-  float* vout = val ? val + r * k : nullptr;
-
+  // (the whole cluster takes this branch alike: it depends on the row only)
   if (n <= k) {
-    for (int j = threadIdx.x; j < k; j += kThreads) {
-      const bool v = j < n;
-      out[j] = v ? j : -1;
-      if (vout) vout[j] = v ? row[j] : __int_as_float(0x7fc00000);
+    if (crank == 0) {
+      for (int j = threadIdx.x; j < k; j += kThreads) {
+        const bool v = j < n;
+        out[j] = v ? j : -1;
+        if (vout) vout[j] = v ? row[j] : __int_as_float(0x7fc00000);
+      }
     }
     return;
   }
 
-  // ---- 1. threshold estimate from evenly spaced samples
-  uint32_t t0 = 0u;
-  if (n > kCap) {
-#pragma unroll
-    for (int q = 0; q < kSamples / kThreads; ++q) {
-      const int s = threadIdx.x + q * kThreads;
-      const int j = static_cast<int>((static_cast<int64_t>(2 * s + 1) * n) / (2 * kSamples));
-      sh.cand_key[(s / (kSamples / kWarps)) * kRegion + s % (kSamples / kWarps)] =
-          order_key(__ldg(row + j));
+  // ---- 1. threshold from evenly spaced samples (identical in every CTA)
+  float fth = -INFINITY;
+  {
+    const int S = n > 32768 ? 4096 : 1024;
+    const int all_fit = C * (CAP - 64);           // no region can overflow below this
+    const int need = max(S, min(2 * k + 64, all_fit));
+    if (n > need) {
+      const int per = S / kWarps;                 // samples per region (<= kRegion)
+      uint32_t mn = 0xffffffffu, mx = 0u;
+      for (int s = threadIdx.x; s < S; s += kThreads) {
+        const int j = static_cast<int>((static_cast<int64_t>(2 * s + 1) * n) / (2 * S));
+        const uint32_t u = order_key(__ldg(row + j));
+        sh.cand_key[(s / per) * kRegion + s % per] = u;
+        mn = min(mn, u);
+        mx = max(mx, u);
+      }
+      if (lane == 0) sh.wcnt[warp] = per;
+      cluster_minmax<1>(mn, mx, sh);
+      const float expect = static_cast<float>(S) * k / n;
+      const int r0 = static_cast<int>(ceilf(expect + 4.f * sqrtf(expect) + 8.f));
+      if (r0 < S) {
+        // two histogram levels: the bin of the r0-th largest sample, then
+        // the same inside that bin, so the edge lies within 2^(shift-11)
+        // keys of the sample itself (a coarse edge would let many more
+        // scores through than the margin allows)
+        const uint32_t lo = sh.red_min;
+        const int shift = bin_shift(lo, sh.red_max);
+        hist_cut<1>(RegionKeys<CAP>{&sh}, static_cast<uint32_t>(r0), lo, shift, sh);
+        const uint32_t b1 = sh.sel_digit;
+        uint32_t t0 = lo + (b1 << shift);
+        if (shift > 0) {
+          const uint32_t r1 = static_cast<uint32_t>(r0) - sh.cnt_above;
+          const int shift2 = shift > kBinBits ? shift - kBinBits : 0;
+          hist_cut<1>(BinKeys<RegionKeys<CAP>>{RegionKeys<CAP>{&sh}, lo, shift, b1}, r1, t0,
+                      shift2, sh);
+          t0 += sh.sel_digit << shift2;
+        }
+        fth = key_float(t0);
+      }
+      __syncthreads();   // the samples are overwritten below
     }
-    if (lane == 0) sh.wcnt[warp] = kSamples / kWarps;
-    __syncthreads();
-    const float expect = static_cast<float>(kSamples) * k / n;
-    const int r0 = static_cast<int>(ceilf(expect + 4.f * sqrtf(expect) + 8.f));
-    if (r0 < kSamples) {
-      uint32_t unused;
-      t0 = select_kth(RegionKeys{&sh}, static_cast<uint32_t>(r0), unused, sh);
-    }
-    __syncthreads();   // the samples are overwritten below
   }
 
-  // ---- 2. filter: warp w appends the keys >= t0 of its eighth of the row
+  // ---- 2. filter: warp w of rank c appends the passing scores of segment 8c + w
+  uint32_t cmn = 0xffffffffu, cmx = 0u;
   {
     const int n4 = n >> 2;
-    const int seg = (n4 + kWarps - 1) / kWarps;
-    const int f0 = min(warp * seg, n4), f1 = min(f0 + seg, n4);
+    const int gw = static_cast<int>(crank) * kWarps + warp;
+    const int seg = (n4 + C * kWarps - 1) / (C * kWarps);
+    const int f0 = min(gw * seg, n4), f1 = min(f0 + seg, n4);
     uint32_t* rk = sh.cand_key + warp * kRegion;
     int32_t* rp = sh.cand_pos + warp * kRegion;
     const float4* row4 = reinterpret_cast<const float4*>(row);
@@ -310,45 +518,137 @@ __global__ void __launch_bounds__(kThreads, 3)
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int j4 = base + u * 32 + lane;
-        const uint32_t key[4] = {order_key(v[u].x), order_key(v[u].y), order_key(v[u].z),
-                                 order_key(v[u].w)};
+        const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
         uint32_t flags = 0;
         if (j4 < f1) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) flags |= (key[e] >= t0 ? 1u : 0u) << e;
+          for (int e = 0; e < 4; ++e) flags |= (x[e] >= fth ? 1u : 0u) << e;
         }
-        cnt = region_append(rk, rp, cnt, key, flags, 4 * j4);
+        if (__any_sync(0xffffffffu, flags != 0))
+          cnt = region_append<CAP>(rk, rp, cnt, x, flags, 4 * j4, cmn, cmx);
       }
     }
-    if (warp == kWarps - 1) {           // ragged tail: the last warp's region comes last
+    if (gw == C * kWarps - 1) {         // ragged tail: the last segment's region comes last
       const int j = 4 * n4 + lane;
-      uint32_t key[4] = {0u, 0u, 0u, 0u};
+      float x[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t flags = 0;
       if (lane < 4 && j < n) {
-        key[0] = order_key(__ldg(row + j));
-        flags = key[0] >= t0 ? 1u : 0u;
+        x[0] = __ldg(row + j);
+        flags = x[0] >= fth ? 1u : 0u;
       }
-      // one key per lane: positions j = 4*n4 + lane
-      cnt = region_append(rk, rp, cnt, key, flags, j);
+      cnt = region_append<CAP>(rk, rp, cnt, x, flags, j, cmn, cmx);
     }
     if (lane == 0) sh.wcnt[warp] = cnt;
   }
   __syncthreads();
-  uint32_t m = 0;
-  bool overflow = false;
+  uint32_t m = 0, overflow = 0;
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) {
     m += sh.wcnt[w];
-    overflow |= sh.wcnt[w] > static_cast<uint32_t>(kRegion);
+    overflow |= sh.wcnt[w] > static_cast<uint32_t>(kRegion) ? 1u : 0u;
+  }
+  if constexpr (C > 1) {
+    if (threadIdx.x == 0) {
+      sh.xch[kXCand] = m;
+      sh.xch[kXOverflow] = overflow;
+    }
+    Cluster<C>::sync();
+    gather_xch<C>(sh);
+    m = 0;
+    overflow = 0;
+    for (unsigned q = 0; q < C; ++q) {
+      m += sh.xall[q][kXCand];
+      overflow |= sh.xall[q][kXOverflow];
+    }
+    Cluster<C>::sync();   // xch is read before it is written again
   }
   if (overflow || m < static_cast<uint32_t>(k)) {
-    topk_row_global(row, n, k, out, vout, sh);
+    if (crank == 0) topk_row_global(row, n, k, out, vout, sh);
     return;
   }
 
-  // ---- 3. exact k-th key among the candidates
-  uint32_t krem;
-  const uint32_t T = select_kth(RegionKeys{&sh}, static_cast<uint32_t>(k), krem, sh);
+  // ---- 3. exact k-th key: two histogram cuts, then the fine bin's keys ranked
+  cluster_minmax<C>(cmn, cmx, sh);
+  uint32_t lo = sh.red_min;
+  int shift = bin_shift(lo, sh.red_max);
+  hist_cut<C>(RegionKeys<CAP>{&sh}, static_cast<uint32_t>(k), lo, shift, sh);
+  uint32_t bsel = sh.sel_digit;
+  uint32_t kk = static_cast<uint32_t>(k) - sh.cnt_above;   // rank inside the cut bin
+  if (shift > 0) {
+    // the candidates can span many binades (a row whose k-th score is
+    // negative spans the sign), so the first cut can be coarse: cut again
+    // inside its bin
+    const uint32_t lo2 = lo + (bsel << shift);
+    const int shift2 = shift > kBinBits ? shift - kBinBits : 0;
+    hist_cut<C>(BinKeys<RegionKeys<CAP>>{RegionKeys<CAP>{&sh}, lo, shift, bsel}, kk, lo2, shift2,
+                sh);
+    bsel = sh.sel_digit;
+    kk -= sh.cnt_above;
+    lo = lo2;
+    shift = shift2;
+  }
+  uint32_t T, krem;
+  if (shift == 0) {
+    // every key of the bin is the same key
+    T = lo + bsel;
+    krem = kk;
+  } else {
+    // gather this CTA's keys of the cut bin
+    if (threadIdx.x == 0) sh.list_n = 0;
+    __syncthreads();
+    RegionKeys<CAP>{&sh}.for_each([&](uint32_t u) {
+      if (((u - lo) >> shift) == bsel) {
+        const uint32_t i = atomicAdd(&sh.list_n, 1u);
+        if (i < static_cast<uint32_t>(kList)) sh.list_key[i] = u;
+      }
+    });
+    __syncthreads();
+    uint32_t total = sh.list_n;
+    const uint32_t* lk = sh.list_key;
+    if constexpr (C > 1) {
+      if (threadIdx.x == 0) sh.xch[kXList] = sh.list_n;
+      Cluster<C>::sync();
+      gather_xch<C>(sh);
+      total = 0;
+      for (unsigned q = 0; q < C; ++q) total += sh.xall[q][kXList];
+      if (total <= static_cast<uint32_t>(kList)) {
+        // copy the cluster's keys of the bin into this CTA, in rank order
+        for (uint32_t i = threadIdx.x; i < total; i += kThreads) {
+          uint32_t off = i;
+          unsigned q = 0;
+          while (off >= sh.xall[q][kXList]) off -= sh.xall[q][kXList], ++q;
+          sh.mlist[i] = Cluster<C>::at(sh.list_key, q)[off];
+        }
+      }
+      Cluster<C>::sync();   // every CTA has its copy before any list is reused
+      lk = sh.mlist;
+    }
+    if (total > static_cast<uint32_t>(kList)) {
+      // too many keys share the cut bin (massive ties): exact fallback
+      if (crank == 0) topk_row_global(row, n, k, out, vout, sh);
+      return;
+    }
+    // rank every key of the bin against all of them: the kk-th largest is the
+    // key with fewer than kk keys above it and at least kk at or above it
+    if (threadIdx.x == 0) sh.res_key = 0u;
+    __syncthreads();
+    for (uint32_t i = threadIdx.x; i < total; i += kThreads) {
+      const uint32_t own = lk[i];
+      uint32_t gt = 0, ge = 0;
+      for (uint32_t j = 0; j < total; ++j) {
+        const uint32_t v = lk[j];
+        gt += v > own ? 1u : 0u;
+        ge += v >= own ? 1u : 0u;
+      }
+      if (gt < kk && ge >= kk) {
+        sh.res_key = own;
+        sh.res_rem = kk - gt;
+      }
+    }
+    __syncthreads();
+    T = sh.res_key;
+    krem = sh.res_rem;
+  }
 
   // ---- 4. ordered output: keys > T, and the first krem keys == T
   {
@@ -369,6 +669,24 @@ __global__ void __launch_bounds__(kThreads, 3)
     }
     __syncthreads();
     uint32_t tie_before = 0, out_before = 0;
+    if constexpr (C > 1) {
+      if (threadIdx.x == 0) {
+        uint32_t g = 0, e = 0;
+        for (int w = 0; w < kWarps; ++w) {
+          g += sh.wsum2[w];
+          e += sh.wsum[w];
+        }
+        sh.xch[kXGt] = g;
+        sh.xch[kXEq] = e;
+      }
+      Cluster<C>::sync();
+      gather_xch<C>(sh);
+      for (unsigned q = 0; q < crank; ++q) {
+        const uint32_t room = krem > tie_before ? krem - tie_before : 0u;
+        out_before += sh.xall[q][kXGt] + min(sh.xall[q][kXEq], room);
+        tie_before += sh.xall[q][kXEq];
+      }
+    }
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
       if (w < warp) {
@@ -396,6 +714,105 @@ __global__ void __launch_bounds__(kThreads, 3)
       tie_before += __popc(eqb);
     }
   }
+  // the next row (or, in a cluster, the other CTAs) may reuse shared memory
+  if constexpr (C > 1) Cluster<C>::sync();
+  else __syncthreads();
+}
+
+struct RowInfo {
+  const float* row;
+  int n;
+};
+
+__device__ __forceinline__ RowInfo row_info(int64_t r, const float* logits, int64_t ld,
+                                            const int32_t* cu_q, const int32_t* cu_k, int B) {
+  int lo = 0, hi = B;  // cu_q[lo] <= r < cu_q[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(cu_q + mid) <= r) lo = mid; else hi = mid;
+  }
+  const int len_q = __ldg(cu_q + lo + 1) - __ldg(cu_q + lo);
+  const int len_k = __ldg(cu_k + lo + 1) - __ldg(cu_k + lo);
+  const int i = static_cast<int>(r - __ldg(cu_q + lo));
+  RowInfo ri;
+  ri.row = logits + r * ld;
+  ri.n = len_k - len_q + i + 1;  // candidates 0..p
+  return ri;
+}
+
+// Pulls a score row towards L2 (16-byte granules; the tail below 16 bytes is
+// read normally).
+__device__ __forceinline__ void prefetch_row(const float* row, int n) {
+  const uint32_t bytes = static_cast<uint32_t>(n) * 4u & ~15u;
+  for (uint32_t off = 0; off < bytes; off += 32768u)
+    prefetch_l2_bulk(reinterpret_cast<const uint8_t*>(row) + off, min(32768u, bytes - off));
+}
+
+// C == 1: a persistent grid; CTA b takes rows b, b + grid, ... and pulls its
+// next row into L2 at the start of each row.  C > 1: one row per cluster.
+template <int C, int CAP>
+__global__ void __launch_bounds__(kThreads, C == 1 ? (CAP <= 5120 ? 4 : 2) : 1)
+    topk_kernel(const float* __restrict__ logits, int64_t ld, const int32_t* __restrict__ cu_q,
+                const int32_t* __restrict__ cu_k, int B, int64_t total_q, int k,
+                int32_t* __restrict__ idx, float* __restrict__ val) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  Shared<CAP>& sh = *reinterpret_cast<Shared<CAP>*>(smem_raw);
+  if constexpr (C == 1) {
+    int64_t r = blockIdx.x;
+    if (r >= total_q) return;
+    RowInfo cur = row_info(r, logits, ld, cu_q, cu_k, B);
+    if (threadIdx.x == 0) prefetch_row(cur.row, cur.n);
+    for (; r < total_q; r += gridDim.x) {
+      const int64_t rn = r + gridDim.x;
+      RowInfo nxt = cur;
+      if (rn < total_q) {
+        nxt = row_info(rn, logits, ld, cu_q, cu_k, B);
+        if (threadIdx.x == 0) prefetch_row(nxt.row, nxt.n);
+      }
+      topk_row<1, CAP>(cur.row, cur.n, k, idx + r * k, val ? val + r * k : nullptr, sh);
+      cur = nxt;
+    }
+  } else {
+    const int64_t r = blockIdx.x / C;
+    const RowInfo ri = row_info(r, logits, ld, cu_q, cu_k, B);
+    topk_row<C, CAP>(ri.row, ri.n, k, idx + r * k, val ? val + r * k : nullptr, sh);
+  }
+}
+
+template <int C, int CAP>
+cudaError_t launch_t(const TopkArgs& a, cudaStream_t s) {
+  const size_t smem = sizeof(Shared<CAP>);
+  auto kern = topk_kernel<C, CAP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  int64_t grid = a.total_q * C;
+  if (C == 1) {
+    int dev = 0, sms = 148, per_sm = 1;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) !=
+            cudaSuccess || per_sm < 1)
+      per_sm = 1;
+    const int64_t cap = static_cast<int64_t>(sms) * per_sm;
+    if (grid > cap) grid = cap;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = C > 1 ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, kern, a.logits, a.ld, a.cu_q, a.cu_k, a.B, a.total_q, a.k, a.idx,
+                         a.val);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -403,13 +820,12 @@ __global__ void __launch_bounds__(kThreads, 3)
 cudaError_t launch_topk(const TopkArgs& a, DevErr err, cudaStream_t s) {
   (void)err;
   if (a.total_q == 0) return cudaSuccess;
-  const size_t smem = sizeof(Shared);
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  topk_kernel<<<static_cast<unsigned>(a.total_q), kThreads, smem, s>>>(
-      a.logits, a.ld, a.cu_q, a.cu_k, a.B, a.k, a.idx, a.val);
-  return cudaGetLastError();
+  // A row per CTA fills the GPU when there are enough rows; a few long rows
+  // (a decode batch) are each split over a cluster of CTAs.
+  const bool split = a.total_q < 148 && a.max_len_k > 16384 && a.k <= 2048;
+  if (split) return launch_t<kSplitC, 5120>(a, s);
+  if (a.k <= 2048) return launch_t<1, 5120>(a, s);
+  return launch_t<1, 8192>(a, s);
 }
 
 }  // namespace dsa
