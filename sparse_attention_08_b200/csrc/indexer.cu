@@ -42,6 +42,8 @@ namespace {
 
 constexpr int kBlockK = 128;      // keys per tile (MMA M)
 constexpr int kKbPerItem = 16;    // key blocks per work item
+constexpr int kDenseKb = 8;       // key blocks per work item of a one-query batch
+constexpr int kMaxDenseB = 2048;  // sequences a one-query batch may have for the dense list
 constexpr int kStages = 6;        // key-tile pipeline depth
 constexpr int kEpiThreads = 128;   // one epilogue warpgroup
 
@@ -57,6 +59,7 @@ struct Params {
   int n_qg;   // query groups per sequence (virtual)
   int n_kc;   // key chunks per sequence (virtual)
   int64_t n_items;
+  int dense;  // 1: one query per sequence; items are the real (sequence, key chunk) pairs
   DevErr err;
 };
 
@@ -70,13 +73,9 @@ struct Item {
   int nkb;      // key blocks in the item
 };
 
+// The item of sequence b, query group qg, key chunk kc of kb key blocks.
 template <int QPT>
-__device__ __forceinline__ bool decode_item(int64_t item, const Params& P, Item& it) {
-  const int kc = static_cast<int>(item % P.n_kc);
-  const int64_t rest = item / P.n_kc;
-  const int qg = static_cast<int>(rest % P.n_qg);
-  const int b = static_cast<int>(rest / P.n_qg);
-  if (b >= P.B) return false;
+__device__ __forceinline__ bool fill_item(int b, int qg, int kc, int kb, const Params& P, Item& it) {
   const int cq0 = __ldg(P.cu_q + b), cq1 = __ldg(P.cu_q + b + 1);
   const int ck0 = __ldg(P.cu_k + b), ck1 = __ldg(P.cu_k + b + 1);
   it.len_q = cq1 - cq0;
@@ -85,14 +84,39 @@ __device__ __forceinline__ bool decode_item(int64_t item, const Params& P, Item&
   if (it.q0 >= it.len_q || it.len_q > it.len_k) return false;
   it.nq = min(QPT, it.len_q - it.q0);
   const int p_max = it.len_k - it.len_q + it.q0 + it.nq - 1;
-  const int kbeg = kc * kKbPerItem * kBlockK;
-  const int kend = min(kbeg + kKbPerItem * kBlockK, p_max + 1);
+  const int kbeg = kc * kb * kBlockK;
+  const int kend = min(kbeg + kb * kBlockK, p_max + 1);
   if (kbeg >= kend) return false;
   it.kb0 = kbeg / kBlockK;
   it.nkb = (kend - kbeg + kBlockK - 1) / kBlockK;
   it.q_row0 = cq0 + it.q0;
   it.k_row0 = ck0;
   return true;
+}
+
+// Item number -> item.  Prefill and chunk batches use a virtual item space
+// (sequence, query group, key chunk) in which items outside the causal
+// triangle are skipped.  One-query batches (decode) list only their real
+// (sequence, key chunk) pairs: pre[b] counts the chunks of the sequences
+// before b, so the persistent grid's stride deals out equal shares of work
+// whatever the mix of cache lengths.
+template <int QPT>
+__device__ __forceinline__ bool decode_item(int64_t item, const Params& P, const int* pre,
+                                            Item& it) {
+  if (QPT == 1 && P.dense) {
+    int lo = 0, hi = P.B;   // pre[lo] <= item < pre[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pre[mid] <= item) lo = mid; else hi = mid;
+    }
+    return fill_item<QPT>(lo, 0, static_cast<int>(item - pre[lo]), kDenseKb, P, it);
+  }
+  const int kc = static_cast<int>(item % P.n_kc);
+  const int64_t rest = item / P.n_kc;
+  const int qg = static_cast<int>(rest % P.n_qg);
+  const int b = static_cast<int>(rest / P.n_qg);
+  if (b >= P.B) return false;
+  return fill_item<QPT>(b, qg, kc, kKbPerItem, P, it);
 }
 
 // NT = MMA N = queries per tile * H_I: 256 (four queries of 64 heads) for
@@ -121,7 +145,8 @@ struct Layout {
   // barriers: q_full[2], q_empty[2], k_full[S], k_empty[S], acc_full[B], acc_empty[B], drain
   static constexpr uint32_t kNumBars = 2 + 2 + kStages + kStages + 2 * kBufs + 1;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr uint32_t kBytes = kOffMisc + 16;
+  static constexpr uint32_t kOffPre = kOffMisc + 16;     // int32 [kMaxDenseB + 1]
+  static constexpr uint32_t kBytes = kOffPre + (kMaxDenseB + 1) * 4;
   static constexpr uint32_t kSmem = kBytes + 1024;      // + alignment slack
   static constexpr uint32_t kSwizzle = D_I == 128 ? kSwizzle128B : kSwizzle64B;
   static constexpr uint32_t kSbo = 8 * D_I;              // 8 rows of one swizzle width
@@ -151,9 +176,36 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
   const uint32_t drain_bar = bar0 + 8u * (4 + 2 * kStages + 2 * kBufs);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
+  int* pre = reinterpret_cast<int*>(smem + L::kOffPre);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
+
+  // one-query batches: chunk counts of the sequences, prefix-summed by warp 0
+  // (made visible to every role by the barrier after the TMEM allocation)
+  int64_t n_items = P.n_items;
+  if (QPT == 1 && P.dense) {
+    if (warp == 0) {
+      int carry = 0;
+      for (int b0 = 0; b0 < P.B; b0 += 32) {
+        const int b = b0 + lane;
+        int c = 0;
+        if (b < P.B && __ldg(P.cu_q + b + 1) > __ldg(P.cu_q + b)) {
+          const int len_k = __ldg(P.cu_k + b + 1) - __ldg(P.cu_k + b);
+          c = (len_k + kDenseKb * kBlockK - 1) / (kDenseKb * kBlockK);
+        }
+        int x = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        if (b < P.B) pre[b] = carry + x - c;
+        carry += __shfl_sync(0xffffffffu, x, 31);
+      }
+      if (lane == 0) pre[P.B] = carry;
+    }
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -182,6 +234,7 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (QPT == 1 && P.dense) n_items = pre[P.B];
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -189,9 +242,12 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
       int64_t qc = 0, kc = 0;
       bool ok = true;
       const bool dropped = (P.err.inject & kInjectDropFirstKeyLoad) != 0;
-      for (int64_t item = blockIdx.x; ok && item < P.n_items; item += gridDim.x) {
+      // the key tiles are read by every query group: keep them in L2 while
+      // the score rows stream through it
+      const uint64_t keep = l2_policy_evict_last();
+      for (int64_t item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
         Item it;
-        if (!decode_item<QPT>(item, P, it)) continue;
+        if (!decode_item<QPT>(item, P, pre, it)) continue;
         const int qb = static_cast<int>(qc & 1);
         if (!(ok = mbar_wait(q_empty(qb), static_cast<uint32_t>(((qc >> 1) & 1) ^ 1), P.err))) break;
         mbar_arrive_expect_tx(q_full(qb), L::kQBytes);
@@ -205,8 +261,8 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
           // issuer's bounded wait for it runs out
           if (kc != 0 || !dropped) {
             mbar_arrive_expect_tx(k_full(st), L::kKBytes);
-            tma_load_2d(sbase + L::kOffK + st * L::kKBytes, &tmap_k, 0,
-                        it.k_row0 + (it.kb0 + j) * kBlockK, k_full(st));
+            tma_load_2d_hint(sbase + L::kOffK + st * L::kKBytes, &tmap_k, 0,
+                             it.k_row0 + (it.kb0 + j) * kBlockK, k_full(st), keep);
           }
           ++kc;
         }
@@ -235,9 +291,9 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
     bool ok = true;
     const uint64_t a0 = smem_desc(sbase + L::kOffK, 16, L::kSbo, L::kSwizzle);
     const uint64_t b0 = smem_desc(sbase + L::kOffQ, 16, L::kSbo, L::kSwizzle);
-    for (int64_t item = blockIdx.x; ok && item < P.n_items; item += gridDim.x) {
+    for (int64_t item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
       Item it;
-      if (!decode_item<QPT>(item, P, it)) continue;
+      if (!decode_item<QPT>(item, P, pre, it)) continue;
       const int qb = static_cast<int>(qc & 1);
       if (!(ok = warp_wait(q_full(qb), static_cast<uint32_t>((qc >> 1) & 1), P.err))) break;
       const uint64_t bq = b0 + ((static_cast<uint32_t>(qb) * L::kQBytes) >> 4);
@@ -295,9 +351,9 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
     float* wq = wq_s + eg * kHalf;
     int64_t ac = 0;
     bool ok = true;
-    for (int64_t item = blockIdx.x; item < P.n_items; item += gridDim.x) {
+    for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
       Item it;
-      if (!decode_item<QPT>(item, P, it)) continue;
+      if (!decode_item<QPT>(item, P, pre, it)) continue;
       // the warpgroup stops together once a wait of one of its warps gave up
       if (named_bar_or(bar_id, kEpiThreads, !ok)) break;
       // head weights of this half of the query group: w * q_scale
@@ -342,6 +398,13 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
 #pragma unroll
           for (int u = 0; u < kChunksPerWait; ++u) tmem_ld_32x32b_x32(dcol + (cg + u) * 32, v[u]);
           tmem_wait_ld();
+          if (cg + kChunksPerWait >= kHalf / 32) {
+            // the last columns are in registers: hand the buffer back before
+            // they are folded, so the next MMA into it can start earlier
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty(ab));
+          }
 #pragma unroll
           for (int u = 0; u < kChunksPerWait; ++u) {
 #pragma unroll
@@ -359,9 +422,6 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
             }
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(acc_empty(ab));
         if (s_local < it.len_k) {
           const int p0 = it.len_k - it.len_q + it.q0;
 #pragma unroll
@@ -371,7 +431,8 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
 #pragma unroll
             for (int ch = 0; ch < NCH; ++ch) sum += acc[ql][ch].x + acc[ql][ch].y;
             if (qi < it.nq && s_local <= p0 + qi)
-              P.logits[static_cast<int64_t>(it.q_row0 + qi) * P.ld + s_local] = sum * ks;
+              st_global_stream(P.logits + static_cast<int64_t>(it.q_row0 + qi) * P.ld + s_local,
+                               sum * ks);
           }
         }
       }
@@ -399,6 +460,7 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const Indexer
   P.logits = a.logits;
   P.ld = a.ld;
   P.B = a.B;
+  P.dense = (L::QPT == 1 && a.max_len_q <= 1 && a.B <= kMaxDenseB) ? 1 : 0;
   P.n_qg = (a.max_len_q + L::QPT - 1) / L::QPT;
   P.n_kc = (a.max_len_k + kKbPerItem * kBlockK - 1) / (kKbPerItem * kBlockK);
   P.n_items = static_cast<int64_t>(a.B) * P.n_qg * P.n_kc;

@@ -167,6 +167,30 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, 
       : "memory");
 }
 
+// An L2 cache policy that keeps lines in L2 ahead of others (for data that is
+// read again and again while a large stream passes through L2).
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// As tma_load_2d, with an L2 cache policy for the lines it reads.
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* m, int32_t x,
+                                                 int32_t y, uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+// A 4-byte store that streams past the caches (evict-first): results that
+// nothing on this SM reads again should not push reused data out of L2.
+__device__ __forceinline__ void st_global_stream(float* p, float v) {
+  asm volatile("st.global.cs.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // cp.async (LDGSTS): 16-byte global -> shared copies, cached in L2 only.
 // ---------------------------------------------------------------------------

@@ -751,7 +751,7 @@ __device__ __forceinline__ void prefetch_row(const float* row, int n) {
 // C == 1: a persistent grid; CTA b takes rows b, b + grid, ... and pulls its
 // next row into L2 at the start of each row.  C > 1: one row per cluster.
 template <int C, int CAP>
-__global__ void __launch_bounds__(kThreads, C == 1 ? (CAP <= 5120 ? 4 : 2) : 1)
+__global__ void __launch_bounds__(kThreads, C == 1 ? (CAP <= 5120 ? 4 : 2) : 4)
     topk_kernel(const float* __restrict__ logits, int64_t ld, const int32_t* __restrict__ cu_q,
                 const int32_t* __restrict__ cu_k, int B, int64_t total_q, int k,
                 int32_t* __restrict__ idx, float* __restrict__ val) {
