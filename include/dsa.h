@@ -272,6 +272,40 @@ DSA_API dsa_status_t dsa_indexer_kl(const void* q, const void* kv, const int32_t
 DSA_API size_t dsa_indexer_kl_workspace_size(int64_t total_q, int H, int k);
 
 /*
+ * The indexer's backward ("DeepSeek V3.2 and the lightning indexer", section
+ * "Teaching a dense model to be sparse": in the warm-up only the indexer is
+ * trained, on the KL signal its scores get; dsa_indexer_kl gives the gradient
+ * of that loss with respect to the scores).  With qhat = q8 * q_scale and
+ * khat = k8 * k_scale (dequantised) and the scores
+ *   I[t,s] = sum_j w[t,j] * ReLU(qhat[t,j,:] . khat[s,:]),   s <= p(t),
+ * and an upstream gradient g[t,s] = dL/dI[t,s], it writes
+ *   dq[t,j,:] = dL/dqhat[t,j,:] = w[t,j] * sum_s g[t,s] [qhat.khat > 0] khat[s,:]
+ *   dw[t,j]   = dL/dw[t,j]      = sum_s g[t,s] ReLU(qhat[t,j,:] . khat[s,:])
+ *   dk[s,:]   = dL/dkhat[s,:]   = sum_{t,j} g[t,s] [qhat.khat > 0] w[t,j] qhat[t,j,:]
+ * (gradients with respect to the dequantised values: the quantisation is
+ * passed straight through; the ReLU's derivative is taken as 0 at 0).
+ *
+ *  q_fp8, q_scale, w, k_fp8, k_scale: as for dsa_indexer_logits (device)
+ *  g        (device) f32 [total_q, ld_g], row = query, column = sequence-local
+ *           key; entries past p are ignored.  ld_g >= max_len_k, multiple of 4.
+ *  dq       (device) f32 [total_q, H_I, d_I]; dw (device) f32 [total_q, H_I];
+ *  dk       (device) f32 [total_k, d_I] (overwritten: the call zeroes it, then
+ *           adds every query's share; keys no query sees get 0).
+ *  Supported: H_I = 64, d_I = 128.
+ *  Arithmetic: the gates from the FP8 tensor-core products; the gated sums on
+ *  the bf16 tensor cores (gradient, scales and weights folded into one bf16
+ *  operand, the e4m3 codes exact in the other), fp32 accumulation.
+ */
+DSA_API dsa_status_t dsa_indexer_backward(const void* q_fp8, const float* q_scale,
+                                          const float* w, const void* k_fp8,
+                                          const float* k_scale, const float* g, int64_t ld_g,
+                                          const int32_t* cu_seqlens_q,
+                                          const int32_t* cu_seqlens_k, int B, int max_len_q,
+                                          int max_len_k, int64_t total_q, int64_t total_k,
+                                          int H_I, int d_I, float* dq, float* dw, float* dk,
+                                          void* stream);
+
+/*
  * The masked MHA mode ("DeepSeek-V3.2" atlas entry, "Design overview" and
  * "Inference efficiency": short prompts are prefilled with a masked MHA
  * standing in for DSA; the pages give no

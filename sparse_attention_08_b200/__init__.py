@@ -17,7 +17,7 @@ __all__ = [
     "dsa_forward_workspace_size", "dsa_get_device_error", "dsa_forward_noalloc",
     "dsa_forward_host", "dsa_forward_host_workspace_size", "dsa_indexer_kl",
     "dsa_indexer_kl_workspace_size", "dsa_masked_mha_fwd", "dsa_masked_mha_workspace_size",
-    "dsa_debug_fault_injection", "EXPORTED",
+    "dsa_debug_fault_injection", "dsa_indexer_backward", "EXPORTED",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -30,7 +30,7 @@ EXPORTED = (
     "dsa_forward_workspace_size", "dsa_status_string", "dsa_get_device_error", "dsa_version",
     "dsa_forward_noalloc", "dsa_forward_host", "dsa_forward_host_workspace_size",
     "dsa_indexer_kl", "dsa_indexer_kl_workspace_size", "dsa_masked_mha_fwd",
-    "dsa_masked_mha_workspace_size", "dsa_debug_fault_injection",
+    "dsa_masked_mha_workspace_size", "dsa_debug_fault_injection", "dsa_indexer_backward",
 )
 
 STATUS = {
@@ -90,6 +90,9 @@ def load():
     lib.dsa_status_string.restype = ctypes.c_char_p
     lib.dsa_get_device_error.argtypes = [P]
     lib.dsa_get_device_error.restype = I
+    lib.dsa_indexer_backward.argtypes = [P, P, P, P, P, P, I64, P, P, I, I, I, I64, I64, I, I, P,
+                                         P, P, P]
+    lib.dsa_indexer_backward.restype = I
     lib.dsa_debug_fault_injection.argtypes = [ctypes.c_uint64, I]
     lib.dsa_debug_fault_injection.restype = None
     lib.dsa_version.argtypes = []
@@ -166,6 +169,34 @@ def dsa_indexer_logits(q_fp8, q_scale, w, k_fp8, k_scale, cu_seqlens_q, cu_seqle
                                    int(max_len_k), int(T_q), int(k8.shape[0]), int(H_I), int(d_I),
                                    _ptr(logits), int(ld_logits), _stream(stream))
     _check(rc, "dsa_indexer_logits")
+
+
+def dsa_indexer_backward(q_fp8, q_scale, w, k_fp8, k_scale, g, cu_seqlens_q, cu_seqlens_k, B,
+                         max_len_q, max_len_k, dq, dw, dk, ld_g=None, stream=None):
+    """The indexer's backward: dq [T_q, 64, 128], dw [T_q, 64], dk [T_k, 128]
+    (f32) from the upstream score gradient g (f32, row stride ld_g)."""
+    import torch
+    q8 = q_fp8.view(torch.uint8) if q_fp8.dtype == torch.float8_e4m3fn else q_fp8
+    k8 = k_fp8.view(torch.uint8) if k_fp8.dtype == torch.float8_e4m3fn else k_fp8
+    _need(q8, torch.uint8, "q_fp8", 3)
+    _need(k8, torch.uint8, "k_fp8", 2)
+    for t, n in ((q_scale, "q_scale"), (w, "w"), (k_scale, "k_scale"), (dw, "dw")):
+        _need(t, torch.float32, n)
+    _need(dq, torch.float32, "dq", 3)
+    _need(dk, torch.float32, "dk", 2)
+    _need(cu_seqlens_q, torch.int32, "cu_seqlens_q")
+    _need(cu_seqlens_k, torch.int32, "cu_seqlens_k")
+    if g.dtype != torch.float32 or not g.is_cuda or g.stride(1) != 1:
+        raise ValueError("g must be a CUDA float32 tensor with contiguous rows")
+    if ld_g is None:
+        ld_g = g.stride(0)
+    T_q, H_I, d_I = q8.shape
+    rc = load().dsa_indexer_backward(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale),
+                                     _ptr(g), int(ld_g), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+                                     int(B), int(max_len_q), int(max_len_k), int(T_q),
+                                     int(k8.shape[0]), int(H_I), int(d_I), _ptr(dq), _ptr(dw),
+                                     _ptr(dk), _stream(stream))
+    _check(rc, "dsa_indexer_backward")
 
 
 def dsa_topk(logits, cu_seqlens_q, cu_seqlens_k, B, max_len_q, max_len_k, k, idx_out,

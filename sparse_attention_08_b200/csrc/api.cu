@@ -375,6 +375,56 @@ dsa_status_t dsa_indexer_kl(const void* q, const void* kv, const int32_t* idx, c
       dsa::launch_indexer_kl(a, next_err(dev), static_cast<cudaStream_t>(stream)));
 }
 
+dsa_status_t dsa_indexer_backward(const void* q_fp8, const float* q_scale, const float* w,
+                                  const void* k_fp8, const float* k_scale, const float* g,
+                                  int64_t ld_g, const int32_t* cu_seqlens_q,
+                                  const int32_t* cu_seqlens_k, int B, int max_len_q,
+                                  int max_len_k, int64_t total_q, int64_t total_k, int H_I,
+                                  int d_I, float* dq, float* dw, float* dk, void* stream) {
+  dsa_status_t st = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_len_q, max_len_k, total_q,
+                                 total_k);
+  if (st != DSA_OK) return st;
+  if (!q_fp8 || !q_scale || !w || !k_fp8 || !k_scale || !g || !dq || !dw || !dk)
+    return DSA_ERR_INVALID_ARG;
+  if (H_I != 64 || d_I != 128) return DSA_ERR_UNSUPPORTED;
+  if (ld_g < max_len_k || ld_g < 1) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_fp8) || !aligned16(k_fp8) || !aligned16(g) || (ld_g % 4) != 0 ||
+      !aligned16(dq) || !aligned16(dk))
+    return DSA_ERR_ALIGNMENT;
+  if (total_q * H_I >= (int64_t(1) << 31) || total_k >= (int64_t(1) << 31) ||
+      static_cast<int64_t>(B) * ((max_len_k + 127) / 128) * ((max_len_q + 255) / 256 + 1) >=
+          (int64_t(1) << 31))
+    return DSA_ERR_UNSUPPORTED;
+  if (total_q == 0 || B == 0 || total_k == 0) return DSA_OK;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != DSA_OK) return st;
+  CUtensorMap tq, tk;
+  if ((st = encode_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_fp8, total_q * H_I, d_I, 1, 256, d_I,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != DSA_OK)
+    return st;
+  if ((st = encode_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, k_fp8, total_k, d_I, 1, 128, d_I,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != DSA_OK)
+    return st;
+  dsa::IndexerBwdArgs a;
+  a.g = g;
+  a.ldg = ld_g;
+  a.w = w;
+  a.q_scale = q_scale;
+  a.k_scale = k_scale;
+  a.cu_q = cu_seqlens_q;
+  a.cu_k = cu_seqlens_k;
+  a.B = B;
+  a.max_len_q = max_len_q;
+  a.max_len_k = max_len_k;
+  a.total_k = total_k;
+  a.dq = dq;
+  a.dw = dw;
+  a.dk = dk;
+  const dsa::DevErr eq = next_err(dev);
+  const dsa::DevErr ek = next_err(dev);
+  return from_cuda(dsa::launch_indexer_bwd(tq, tk, a, eq, ek, static_cast<cudaStream_t>(stream)));
+}
+
 size_t dsa_forward_workspace_size(int64_t total_q, int max_len_k, int k) {
   if (total_q < 0 || max_len_k < 0 || k < 1) return 0;
   const int64_t ld = (static_cast<int64_t>(max_len_k) + 3) / 4 * 4;

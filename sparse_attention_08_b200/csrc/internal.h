@@ -89,6 +89,25 @@ struct MaskedMhaArgs {
   float* lse;
 };
 
+struct IndexerBwdArgs {
+  const float* g;        // [total_q, ldg] upstream gradient of the scores
+  int64_t ldg;
+  const float* w;
+  const float* q_scale;
+  const float* k_scale;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int B, max_len_q, max_len_k;
+  int64_t total_k;
+  float* dq;             // [total_q, 64, 128]
+  float* dw;             // [total_q, 64]
+  float* dk;             // [total_k, 128], zeroed by the launcher first
+};
+
+cudaError_t launch_indexer_bwd(const CUtensorMap& tq, const CUtensorMap& tk,
+                               const IndexerBwdArgs& a, DevErr err_q, DevErr err_k,
+                               cudaStream_t s);
+
 cudaError_t launch_masked_mha(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                               const MaskedMhaArgs& a, DevErr err, cudaStream_t s);
 size_t masked_mha_workspace_bytes(int64_t total_q, int max_len_k);

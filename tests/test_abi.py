@@ -73,6 +73,30 @@ def test_indexer_argument_checks_before_device():
         assert call() == CUDA                      # no device: fails loudly
 
 
+def test_indexer_backward_argument_checks_before_device():
+    lib = dsa.load()
+    p = _fake()
+    args = dict(q=p, qs=p, w=p, k=p, ks=p, g=p, ldg=64, cq=p, ck=p, B=1, mlq=64, mlk=64, tq=64,
+                tk=64, H_I=64, d_I=128, dq=p, dw=p, dk=p)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.dsa_indexer_backward(a["q"], a["qs"], a["w"], a["k"], a["ks"], a["g"], a["ldg"],
+                                        a["cq"], a["ck"], a["B"], a["mlq"], a["mlk"], a["tq"],
+                                        a["tk"], a["H_I"], a["d_I"], a["dq"], a["dw"], a["dk"],
+                                        None)
+    assert call(g=None) == INVALID
+    assert call(dk=None) == INVALID
+    assert call(H_I=32) == UNSUPPORTED
+    assert call(d_I=64) == UNSUPPORTED
+    assert call(ldg=32) == INVALID                 # ld_g < max_len_k
+    assert call(ldg=66) == ALIGN
+    assert call(dq=_fake(0x10004)) == ALIGN
+    assert call(tq=0) == OK
+    if not _have_gpu():
+        assert call() == CUDA
+
+
 def test_topk_and_attention_argument_checks():
     lib = dsa.load()
     p = _fake()
