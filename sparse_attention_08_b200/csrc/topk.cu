@@ -7,15 +7,16 @@
 // min(k, n) largest, ties to the lower position, -0.0 == +0.0, written in
 // ascending position order and padded with -1.
 //
-// How: a row is handled by a cluster of C CTAs of 256 threads.  C = 1 when
-// the batch has enough rows to fill the GPU: a persistent grid of a few CTAs
-// per SM walks the rows and pulls each CTA's next row into L2 while it works
-// on the current one.  C = 8 for a few long rows (a decode batch).  Scores
-// map to order-preserving 32-bit keys (larger float -> larger unsigned key,
-// -0 folded into +0).  The row's 16-byte groups are cut into 8C contiguous
-// segments in position order; warp w of cluster rank c owns segment 8c + w
-// and the w-th region of its CTA's candidate buffer, so candidates stay in
-// position order without any sorting.
+// How: scores map to order-preserving 32-bit keys (larger float -> larger
+// unsigned key, -0 folded into +0).  When the batch has enough rows to fill
+// the GPU, a persistent grid of four 256-thread CTAs per SM walks the rows,
+// one CTA per row, and pulls its next row into L2 while it works on the
+// current one.  A few long rows (a decode batch) are split over a cluster of
+// kSplitC CTAs that filter a quarter of the row each and hand their
+// candidates to cluster rank 0, which finishes the row.  The row's 16-byte
+// groups are cut into 8C contiguous segments in position order; warp w of
+// rank c owns segment 8c + w and one region of its CTA's candidate buffer, so
+// candidates stay in position order without any sorting.
 //  1. Threshold.  Rows longer than about 2k (or than the candidate buffers)
 //     draw S evenly spaced samples (S = 1024, or 4096 past 32768 scores).
 //     Two levels of 2048-bin histograms of their keys (over [min, max], then
@@ -27,19 +28,20 @@
 //  2. Filter.  Each warp streams its segment once (16-byte loads), compares
 //     the raw floats with t0 as a float, and appends the (key, position) of
 //     every score that passes to its region in position order (ballot
-//     prefix), tracking the candidates' key range.
+//     prefix), tracking the candidates' key range.  In a cluster every CTA
+//     then stores its regions into rank 0's merge buffer after those of the
+//     lower ranks, which gives one list in position order.
 //  3. Exact k-th key.  Two levels of 2048-bin histograms of the candidates
-//     (over their key range, then inside the bin that holds the k-th largest;
-//     summed over the cluster through distributed shared memory) find a fine
-//     bin holding the k-th largest and how many keys lie above it; the few
-//     keys of that bin are gathered and ranked against each other, which
-//     gives the k-th key T and how many keys equal to T are kept (krem).
+//     (over their key range, then inside the bin that holds the k-th largest)
+//     find a fine bin holding the k-th largest and how many keys lie above
+//     it; the few keys of that bin are ranked against each other, which gives
+//     the k-th key T and how many keys equal to T are kept (krem).
 //  4. Ordered output.  A key is kept if it is > T or one of the first krem
-//     keys == T in position order (tie ranks from prefixes over the cluster's
-//     CTAs and their warps); output slots come from a second prefix.
+//     keys == T in position order (tie ranks from a prefix over the warps'
+//     contiguous shares of the list); output slots come from a second prefix.
 // If the threshold fails (fewer than k candidates, or a region overflows,
-// e.g. rows of massive ties) or the cut bin holds too many keys, rank 0 falls
-// back to exact radix passes over the whole row in global memory and an
+// e.g. rows of massive ties) or the fine bin holds too many keys, one CTA
+// falls back to exact radix passes over the whole row in global memory and an
 // ordered ballot-scan compaction.  Both routes give the same, unique answer.
 // Every decision that changes how many cluster barriers a CTA passes is taken
 // from values that all CTAs of the cluster read alike.
@@ -59,11 +61,11 @@ namespace cg = cooperative_groups;
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kUnroll = 8;                 // 16-byte loads in flight per lane
-constexpr int kSplitC = 8;                 // CTAs per row for few long rows
+constexpr int kSplitC = 4;                 // CTAs per row for few long rows
 constexpr int kBins = 2048;                // histogram bins (11 bits)
 constexpr int kBinBits = 11;
 constexpr int kBinsPerThread = kBins / kThreads;
-constexpr int kList = 512;                 // keys of the cut bin ranked directly
+constexpr int kList = 512;                 // keys of the fine bin ranked directly
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -85,7 +87,7 @@ __device__ __forceinline__ int bin_shift(uint32_t lo, uint32_t hi) {
 }
 
 // Values a CTA shares with the other CTAs of its cluster.
-enum { kXCand = 0, kXOverflow, kXMin, kXMax, kXList, kXGt, kXEq, kXCount };
+enum { kXCand = 0, kXOverflow, kXCount };
 
 template <int CAP>
 struct Shared {
@@ -102,11 +104,10 @@ struct Shared {
   uint32_t res_key, res_rem;
   uint32_t xch[kXCount];
   uint32_t xall[kSplitC][kXCount];   // every CTA's xch, gathered once (clusters)
-  uint32_t tot[kBins / kSplitC];     // cluster totals of the bins this CTA owns
   uint32_t list_key[kList];
-  uint32_t mlist[kList];             // the cluster's cut-bin keys, gathered
   uint32_t cand_key[CAP];
   int32_t cand_pos[CAP];
+  // (clusters: a merge buffer of CAP keys and CAP positions follows)
 };
 
 // Cluster of C CTAs working on one row; with C == 1 a plain CTA.
@@ -127,19 +128,6 @@ struct Cluster {
     else return cg::this_cluster().map_shared_rank(p, r);
   }
 };
-
-// Copies every cluster CTA's xch into sh.xall (after a cluster barrier that
-// follows the writes), with independent remote loads.
-template <int C, int CAP>
-__device__ __forceinline__ void gather_xch(Shared<CAP>& sh) {
-  if constexpr (C > 1) {
-    if (threadIdx.x < C * kXCount) {
-      const unsigned q = threadIdx.x / kXCount, f = threadIdx.x % kXCount;
-      sh.xall[q][f] = Cluster<C>::at(sh.xch, q)[f];
-    }
-    __syncthreads();
-  }
-}
 
 // Block-wide exclusive scan of one value per thread; *total gets the sum.
 template <int CAP>
@@ -166,16 +154,19 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, Shared<CAP>& sh,
   return before + x - v;
 }
 
+// A warp's candidates: cnt (key, position) pairs in position order.
+struct Seg {
+  const uint32_t* key;
+  const int32_t* pos;
+  uint32_t cnt;
+};
+
 // Key sources.  for_each(f) calls f(key) on every key.
-template <int CAP>
-struct RegionKeys {              // the candidate regions (warp w scans region w)
-  const Shared<CAP>* sh;
+struct SegKeys {                 // each warp its own segment
+  Seg seg;
   template <class F>
   __device__ __forceinline__ void for_each(F f) const {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t cnt = sh->wcnt[warp];
-    const uint32_t* keys = sh->cand_key + warp * (CAP / kWarps);
-    for (uint32_t i = lane; i < cnt; i += 32) f(keys[i]);
+    for (uint32_t i = threadIdx.x & 31; i < seg.cnt; i += 32) f(seg.key[i]);
   }
 };
 struct RowKeys {                 // a whole score row in global memory
@@ -204,10 +195,9 @@ struct BinKeys {
   }
 };
 
-// The cluster-wide min and max of per-thread key ranges; every thread of
-// every CTA gets the same result in sh.red_min / sh.red_max.
-template <int CC, int CAP>
-__device__ void cluster_minmax(uint32_t mn, uint32_t mx, Shared<CAP>& sh) {
+// The CTA-wide min and max of per-thread key ranges, in sh.red_min / red_max.
+template <int CAP>
+__device__ void block_minmax(uint32_t mn, uint32_t mx, Shared<CAP>& sh) {
   const int lane = threadIdx.x & 31;
   mn = __reduce_min_sync(0xffffffffu, mn);
   mx = __reduce_max_sync(0xffffffffu, mx);
@@ -221,73 +211,26 @@ __device__ void cluster_minmax(uint32_t mn, uint32_t mx, Shared<CAP>& sh) {
     atomicMax(&sh.red_max, mx);
   }
   __syncthreads();
-  if constexpr (CC > 1) {
-    if (threadIdx.x == 0) {
-      sh.xch[kXMin] = sh.red_min;
-      sh.xch[kXMax] = sh.red_max;
-    }
-    Cluster<CC>::sync();
-    gather_xch<CC>(sh);
-    if (threadIdx.x == 0) {
-      uint32_t a = 0xffffffffu, b = 0u;
-      for (unsigned r = 0; r < CC; ++r) {
-        a = min(a, sh.xall[r][kXMin]);
-        b = max(b, sh.xall[r][kXMax]);
-      }
-      sh.red_min = a;
-      sh.red_max = b;
-    }
-    Cluster<CC>::sync();   // every CTA has read xch before it is written again
-  }
 }
 
-// Histogram cut: bins of (key - lo) >> shift over the cluster's keys; finds
-// the bin holding the kk-th largest key (sh.sel_digit) and how many keys lie
-// in higher bins (sh.cnt_above).  kk >= 1 and at most the number of keys.
-template <int CC, int CAP, class Keys>
+// Histogram cut: bins of (key - lo) >> shift over one CTA's keys; finds the
+// bin holding the kk-th largest key (sh.sel_digit) and how many keys lie in
+// higher bins (sh.cnt_above).  kk >= 1 and at most the number of keys.
+template <int CAP, class Keys>
 __device__ void hist_cut(const Keys& keys, uint32_t kk, uint32_t lo, int shift, Shared<CAP>& sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int i = 0; i < kBinsPerThread; ++i) sh.hist[threadIdx.x + i * kThreads] = 0u;
   __syncthreads();
   keys.for_each([&](uint32_t u) { atomicAdd(&sh.hist[(u - lo) >> shift], 1u); });
+  __syncthreads();
   // thread t owns bins kBins-1-8t .. kBins-8-8t, counted from the top down
   uint32_t h[kBinsPerThread];
   uint32_t s = 0;
-  if constexpr (CC > 1) {
-    // CTA q adds up bins q*kBins/CC .. (q+1)*kBins/CC - 1 over the cluster
-    // (thread t one bin, the CC remote loads issued together), then every
-    // CTA reads the totals it scans from their owners
-    static_assert(kBins / CC == kThreads, "one owned bin per thread");
-    Cluster<CC>::sync();                        // every CTA's histogram is complete
-    {
-      const unsigned me = Cluster<CC>::rank();
-      const int b = static_cast<int>(me) * kThreads + static_cast<int>(threadIdx.x);
-      uint32_t v[CC];
 #pragma unroll
-      for (int r = 0; r < CC; ++r) v[r] = Cluster<CC>::at(sh.hist, r)[b];
-      uint32_t t = 0;
-#pragma unroll
-      for (int r = 0; r < CC; ++r) t += v[r];
-      sh.tot[threadIdx.x] = t;
-    }
-    Cluster<CC>::sync();                        // every owner's totals are complete
-    {
-      const int b0 = kBins - 1 - kBinsPerThread * static_cast<int>(threadIdx.x);   // top bin
-      const unsigned owner = static_cast<unsigned>(b0) / kThreads;               // same for all 8
-      const uint32_t* tt = Cluster<CC>::at(sh.tot, owner);
-#pragma unroll
-      for (int i = 0; i < kBinsPerThread; ++i) h[i] = tt[(b0 - i) % kThreads];
-#pragma unroll
-      for (int i = 0; i < kBinsPerThread; ++i) s += h[i];
-    }
-  } else {
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < kBinsPerThread; ++i) {
-      h[i] = sh.hist[kBins - 1 - kBinsPerThread * threadIdx.x - i];
-      s += h[i];
-    }
+  for (int i = 0; i < kBinsPerThread; ++i) {
+    h[i] = sh.hist[kBins - 1 - kBinsPerThread * threadIdx.x - i];
+    s += h[i];
   }
   uint32_t x = s;
 #pragma unroll
@@ -311,8 +254,7 @@ __device__ void hist_cut(const Keys& keys, uint32_t kk, uint32_t lo, int shift, 
       c += h[i];
     }
   }
-  if constexpr (CC > 1) Cluster<CC>::sync();    // no CTA clears its histogram while read
-  else __syncthreads();
+  __syncthreads();
 }
 
 // Exact kk-th largest key by radix passes (kk >= 1, at most the number of
@@ -326,7 +268,7 @@ __device__ uint32_t radix_select(const Keys& keys, uint32_t kk, uint32_t& krem, 
     mn = min(mn, u);
     mx = max(mx, u);
   });
-  cluster_minmax<1>(mn, mx, sh);
+  block_minmax(mn, mx, sh);
   const uint32_t diff = sh.red_min ^ sh.red_max;
   krem = kk;
   if (diff == 0u) return sh.red_max;              // every key is equal
@@ -434,7 +376,126 @@ __device__ __forceinline__ uint32_t region_append(uint32_t* rk, int32_t* rp, uin
   return cnt + __popc(b0) + 2u * __popc(b1) + 4u * __popc(b2);
 }
 
-// One row: the whole pipeline, by every thread of every CTA of the cluster.
+// Steps 3 and 4 on one CTA: each warp holds `seg`, its contiguous share of
+// the row's m >= k candidates (the warps' shares in warp order give every
+// candidate once, in position order); (cmn, cmx) is this thread's part of the
+// candidates' key range.  Writes the k kept positions (and scores) to out.
+template <int CAP>
+__device__ void select_and_output(const float* __restrict__ row, int n, int k,
+                                  int32_t* __restrict__ out, float* __restrict__ vout,
+                                  Shared<CAP>& sh, const Seg seg, uint32_t cmn, uint32_t cmx) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const SegKeys keys{seg};
+
+  // ---- 3. exact k-th key: two histogram cuts, then the fine bin's keys ranked
+  block_minmax(cmn, cmx, sh);
+  uint32_t lo = sh.red_min;
+  int shift = bin_shift(lo, sh.red_max);
+  hist_cut(keys, static_cast<uint32_t>(k), lo, shift, sh);
+  uint32_t bsel = sh.sel_digit;
+  uint32_t kk = static_cast<uint32_t>(k) - sh.cnt_above;   // rank inside the cut bin
+  if (shift > 0) {
+    // the candidates can span many binades (a row whose k-th score is
+    // negative spans the sign), so the first cut can be coarse: cut again
+    // inside its bin
+    const uint32_t lo2 = lo + (bsel << shift);
+    const int shift2 = shift > kBinBits ? shift - kBinBits : 0;
+    hist_cut(BinKeys<SegKeys>{keys, lo, shift, bsel}, kk, lo2, shift2, sh);
+    bsel = sh.sel_digit;
+    kk -= sh.cnt_above;
+    lo = lo2;
+    shift = shift2;
+  }
+  uint32_t T, krem;
+  if (shift == 0) {
+    // every key of the bin is the same key
+    T = lo + bsel;
+    krem = kk;
+  } else {
+    if (threadIdx.x == 0) sh.list_n = 0;
+    __syncthreads();
+    keys.for_each([&](uint32_t u) {
+      if (((u - lo) >> shift) == bsel) {
+        const uint32_t i = atomicAdd(&sh.list_n, 1u);
+        if (i < static_cast<uint32_t>(kList)) sh.list_key[i] = u;
+      }
+    });
+    __syncthreads();
+    const uint32_t total = sh.list_n;
+    if (total > static_cast<uint32_t>(kList)) {
+      // too many keys share the cut bin (massive ties): exact fallback
+      topk_row_global(row, n, k, out, vout, sh);
+      return;
+    }
+    // rank every key of the bin against all of them: the kk-th largest is the
+    // key with fewer than kk keys above it and at least kk at or above it
+    if (threadIdx.x == 0) sh.res_key = 0u;
+    __syncthreads();
+    for (uint32_t i = threadIdx.x; i < total; i += kThreads) {
+      const uint32_t own = sh.list_key[i];
+      uint32_t gt = 0, ge = 0;
+      for (uint32_t j = 0; j < total; ++j) {
+        const uint32_t v = sh.list_key[j];
+        gt += v > own ? 1u : 0u;
+        ge += v >= own ? 1u : 0u;
+      }
+      if (gt < kk && ge >= kk) {
+        sh.res_key = own;
+        sh.res_rem = kk - gt;
+      }
+    }
+    __syncthreads();
+    T = sh.res_key;
+    krem = sh.res_rem;
+  }
+
+  // ---- 4. ordered output: keys > T, and the first krem keys == T
+  uint32_t gt = 0, eq = 0;
+  for (uint32_t c = lane; c < seg.cnt; c += 32) {
+    const uint32_t u = seg.key[c];
+    gt += u > T ? 1u : 0u;
+    eq += u == T ? 1u : 0u;
+  }
+  gt = __reduce_add_sync(0xffffffffu, gt);
+  eq = __reduce_add_sync(0xffffffffu, eq);
+  if (lane == 0) {
+    sh.wsum[warp] = eq;
+    sh.wsum2[warp] = gt;
+  }
+  __syncthreads();
+  uint32_t tie_before = 0, out_before = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    if (w < warp) {
+      const uint32_t room = krem > tie_before ? krem - tie_before : 0u;
+      out_before += sh.wsum2[w] + min(sh.wsum[w], room);
+      tie_before += sh.wsum[w];
+    }
+  }
+  const uint32_t lt = (1u << lane) - 1u;
+  for (uint32_t c0 = 0; c0 < seg.cnt; c0 += 32) {
+    const uint32_t c = c0 + lane;
+    const uint32_t u = c < seg.cnt ? seg.key[c] : 0u;
+    const bool is_gt = c < seg.cnt && u > T;
+    const bool is_eq = c < seg.cnt && u == T;
+    const uint32_t eqb = __ballot_sync(0xffffffffu, is_eq);
+    const bool take = is_gt || (is_eq && tie_before + __popc(eqb & lt) < krem);
+    const uint32_t tb = __ballot_sync(0xffffffffu, take);
+    if (take) {
+      const int j = seg.pos[c];
+      const uint32_t slot = out_before + __popc(tb & lt);
+      out[slot] = j;
+      if (vout) vout[slot] = row[j];
+    }
+    out_before += __popc(tb);
+    tie_before += __popc(eqb);
+  }
+  __syncthreads();   // the next row may reuse shared memory
+}
+
+// One row, by every thread of every CTA of the cluster (C > 1: the merged
+// candidates are finished by rank 0 alone, in the CAP keys and CAP positions
+// that follow its Shared block).
 template <int C, int CAP>
 __device__ void topk_row(const float* __restrict__ row, int n, int k, int32_t* __restrict__ out,
                          float* __restrict__ vout, Shared<CAP>& sh) {
@@ -458,7 +519,8 @@ __device__ void topk_row(const float* __restrict__ row, int n, int k, int32_t* _
   float fth = -INFINITY;
   {
     const int S = n > 32768 ? 4096 : 1024;
-    const int all_fit = C * (CAP - 64);           // no region can overflow below this
+    // below this no region, and no cluster's merged list, can overflow
+    const int all_fit = C == 1 ? CAP - 64 : CAP;
     const int need = max(S, min(2 * k + 64, all_fit));
     if (n > need) {
       const int per = S / kWarps;                 // samples per region (<= kRegion)
@@ -470,8 +532,7 @@ __device__ void topk_row(const float* __restrict__ row, int n, int k, int32_t* _
         mn = min(mn, u);
         mx = max(mx, u);
       }
-      if (lane == 0) sh.wcnt[warp] = per;
-      cluster_minmax<1>(mn, mx, sh);
+      block_minmax(mn, mx, sh);                   // (its barriers publish the samples)
       const float expect = static_cast<float>(S) * k / n;
       const int r0 = static_cast<int>(ceilf(expect + 4.f * sqrtf(expect) + 8.f));
       if (r0 < S) {
@@ -479,16 +540,17 @@ __device__ void topk_row(const float* __restrict__ row, int n, int k, int32_t* _
         // the same inside that bin, so the edge lies within 2^(shift-11)
         // keys of the sample itself (a coarse edge would let many more
         // scores through than the margin allows)
+        const SegKeys samples{Seg{sh.cand_key + warp * kRegion, nullptr,
+                                  static_cast<uint32_t>(per)}};
         const uint32_t lo = sh.red_min;
         const int shift = bin_shift(lo, sh.red_max);
-        hist_cut<1>(RegionKeys<CAP>{&sh}, static_cast<uint32_t>(r0), lo, shift, sh);
+        hist_cut(samples, static_cast<uint32_t>(r0), lo, shift, sh);
         const uint32_t b1 = sh.sel_digit;
         uint32_t t0 = lo + (b1 << shift);
         if (shift > 0) {
           const uint32_t r1 = static_cast<uint32_t>(r0) - sh.cnt_above;
           const int shift2 = shift > kBinBits ? shift - kBinBits : 0;
-          hist_cut<1>(BinKeys<RegionKeys<CAP>>{RegionKeys<CAP>{&sh}, lo, shift, b1}, r1, t0,
-                      shift2, sh);
+          hist_cut(BinKeys<SegKeys>{samples, lo, shift, b1}, r1, t0, shift2, sh);
           t0 += sh.sel_digit << shift2;
         }
         fth = key_float(t0);
@@ -499,13 +561,13 @@ __device__ void topk_row(const float* __restrict__ row, int n, int k, int32_t* _
 
   // ---- 2. filter: warp w of rank c appends the passing scores of segment 8c + w
   uint32_t cmn = 0xffffffffu, cmx = 0u;
+  uint32_t* rk = sh.cand_key + warp * kRegion;
+  int32_t* rp = sh.cand_pos + warp * kRegion;
   {
     const int n4 = n >> 2;
     const int gw = static_cast<int>(crank) * kWarps + warp;
     const int seg = (n4 + C * kWarps - 1) / (C * kWarps);
     const int f0 = min(gw * seg, n4), f1 = min(f0 + seg, n4);
-    uint32_t* rk = sh.cand_key + warp * kRegion;
-    int32_t* rp = sh.cand_pos + warp * kRegion;
     const float4* row4 = reinterpret_cast<const float4*>(row);
     uint32_t cnt = 0;
     for (int base = f0; base < f1; base += 32 * kUnroll) {
@@ -541,182 +603,69 @@ __device__ void topk_row(const float* __restrict__ row, int n, int k, int32_t* _
     if (lane == 0) sh.wcnt[warp] = cnt;
   }
   __syncthreads();
-  uint32_t m = 0, overflow = 0;
+  uint32_t m = 0, overflow = 0, before = 0;
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) {
-    m += sh.wcnt[w];
-    overflow |= sh.wcnt[w] > static_cast<uint32_t>(kRegion) ? 1u : 0u;
+    const uint32_t c = sh.wcnt[w];
+    before += w < warp ? c : 0u;
+    m += c;
+    overflow |= c > static_cast<uint32_t>(kRegion) ? 1u : 0u;
   }
-  if constexpr (C > 1) {
+
+  if constexpr (C == 1) {
+    if (overflow || m < static_cast<uint32_t>(k)) {
+      topk_row_global(row, n, k, out, vout, sh);
+      return;
+    }
+    select_and_output<CAP>(row, n, k, out, vout, sh, Seg{rk, rp, sh.wcnt[warp]}, cmn, cmx);
+  } else {
+    // merge: every CTA stores its regions, in warp order, into rank 0's merge
+    // buffer after those of the lower ranks
     if (threadIdx.x == 0) {
       sh.xch[kXCand] = m;
       sh.xch[kXOverflow] = overflow;
     }
     Cluster<C>::sync();
-    gather_xch<C>(sh);
-    m = 0;
+    if (threadIdx.x < C * kXCount) {
+      const unsigned q = threadIdx.x / kXCount, f = threadIdx.x % kXCount;
+      sh.xall[q][f] = Cluster<C>::at(&sh.xch[f], q)[0];
+    }
+    __syncthreads();
+    uint32_t total = 0;
     overflow = 0;
     for (unsigned q = 0; q < C; ++q) {
-      m += sh.xall[q][kXCand];
+      before += q < crank ? sh.xall[q][kXCand] : 0u;
+      total += sh.xall[q][kXCand];
       overflow |= sh.xall[q][kXOverflow];
     }
-    Cluster<C>::sync();   // xch is read before it is written again
-  }
-  if (overflow || m < static_cast<uint32_t>(k)) {
-    if (crank == 0) topk_row_global(row, n, k, out, vout, sh);
-    return;
-  }
-
-  // ---- 3. exact k-th key: two histogram cuts, then the fine bin's keys ranked
-  cluster_minmax<C>(cmn, cmx, sh);
-  uint32_t lo = sh.red_min;
-  int shift = bin_shift(lo, sh.red_max);
-  hist_cut<C>(RegionKeys<CAP>{&sh}, static_cast<uint32_t>(k), lo, shift, sh);
-  uint32_t bsel = sh.sel_digit;
-  uint32_t kk = static_cast<uint32_t>(k) - sh.cnt_above;   // rank inside the cut bin
-  if (shift > 0) {
-    // the candidates can span many binades (a row whose k-th score is
-    // negative spans the sign), so the first cut can be coarse: cut again
-    // inside its bin
-    const uint32_t lo2 = lo + (bsel << shift);
-    const int shift2 = shift > kBinBits ? shift - kBinBits : 0;
-    hist_cut<C>(BinKeys<RegionKeys<CAP>>{RegionKeys<CAP>{&sh}, lo, shift, bsel}, kk, lo2, shift2,
-                sh);
-    bsel = sh.sel_digit;
-    kk -= sh.cnt_above;
-    lo = lo2;
-    shift = shift2;
-  }
-  uint32_t T, krem;
-  if (shift == 0) {
-    // every key of the bin is the same key
-    T = lo + bsel;
-    krem = kk;
-  } else {
-    // gather this CTA's keys of the cut bin
-    if (threadIdx.x == 0) sh.list_n = 0;
-    __syncthreads();
-    RegionKeys<CAP>{&sh}.for_each([&](uint32_t u) {
-      if (((u - lo) >> shift) == bsel) {
-        const uint32_t i = atomicAdd(&sh.list_n, 1u);
-        if (i < static_cast<uint32_t>(kList)) sh.list_key[i] = u;
+    const bool fits = !overflow && total >= static_cast<uint32_t>(k) &&
+                      total <= static_cast<uint32_t>(CAP);
+    uint32_t* mk = reinterpret_cast<uint32_t*>(&sh + 1);
+    int32_t* mp = reinterpret_cast<int32_t*>(mk + CAP);
+    if (fits) {
+      uint32_t* dk = Cluster<C>::at(mk, 0u) + before;
+      int32_t* dp = Cluster<C>::at(mp, 0u) + before;
+      for (uint32_t c = lane; c < sh.wcnt[warp]; c += 32) {
+        dk[c] = rk[c];
+        dp[c] = rp[c];
       }
-    });
-    __syncthreads();
-    uint32_t total = sh.list_n;
-    const uint32_t* lk = sh.list_key;
-    if constexpr (C > 1) {
-      if (threadIdx.x == 0) sh.xch[kXList] = sh.list_n;
-      Cluster<C>::sync();
-      gather_xch<C>(sh);
-      total = 0;
-      for (unsigned q = 0; q < C; ++q) total += sh.xall[q][kXList];
-      if (total <= static_cast<uint32_t>(kList)) {
-        // copy the cluster's keys of the bin into this CTA, in rank order
-        for (uint32_t i = threadIdx.x; i < total; i += kThreads) {
-          uint32_t off = i;
-          unsigned q = 0;
-          while (off >= sh.xall[q][kXList]) off -= sh.xall[q][kXList], ++q;
-          sh.mlist[i] = Cluster<C>::at(sh.list_key, q)[off];
-        }
-      }
-      Cluster<C>::sync();   // every CTA has its copy before any list is reused
-      lk = sh.mlist;
     }
-    if (total > static_cast<uint32_t>(kList)) {
-      // too many keys share the cut bin (massive ties): exact fallback
-      if (crank == 0) topk_row_global(row, n, k, out, vout, sh);
+    Cluster<C>::sync();   // the merged list is complete; no CTA reads another's memory after
+    if (crank != 0) return;
+    if (!fits) {
+      topk_row_global(row, n, k, out, vout, sh);
       return;
     }
-    // rank every key of the bin against all of them: the kk-th largest is the
-    // key with fewer than kk keys above it and at least kk at or above it
-    if (threadIdx.x == 0) sh.res_key = 0u;
-    __syncthreads();
-    for (uint32_t i = threadIdx.x; i < total; i += kThreads) {
-      const uint32_t own = lk[i];
-      uint32_t gt = 0, ge = 0;
-      for (uint32_t j = 0; j < total; ++j) {
-        const uint32_t v = lk[j];
-        gt += v > own ? 1u : 0u;
-        ge += v >= own ? 1u : 0u;
-      }
-      if (gt < kk && ge >= kk) {
-        sh.res_key = own;
-        sh.res_rem = kk - gt;
-      }
+    const uint32_t share = (total + kWarps - 1) / kWarps;
+    const uint32_t s0 = min(warp * share, total), s1 = min(s0 + share, total);
+    cmn = 0xffffffffu;
+    cmx = 0u;
+    for (uint32_t c = s0 + lane; c < s1; c += 32) {
+      cmn = min(cmn, mk[c]);
+      cmx = max(cmx, mk[c]);
     }
-    __syncthreads();
-    T = sh.res_key;
-    krem = sh.res_rem;
+    select_and_output<CAP>(row, n, k, out, vout, sh, Seg{mk + s0, mp + s0, s1 - s0}, cmn, cmx);
   }
-
-  // ---- 4. ordered output: keys > T, and the first krem keys == T
-  {
-    const uint32_t cnt = sh.wcnt[warp];
-    const uint32_t* rk = sh.cand_key + warp * kRegion;
-    const int32_t* rp = sh.cand_pos + warp * kRegion;
-    uint32_t gt = 0, eq = 0;
-    for (uint32_t c = lane; c < cnt; c += 32) {
-      const uint32_t u = rk[c];
-      gt += u > T ? 1u : 0u;
-      eq += u == T ? 1u : 0u;
-    }
-    gt = __reduce_add_sync(0xffffffffu, gt);
-    eq = __reduce_add_sync(0xffffffffu, eq);
-    if (lane == 0) {
-      sh.wsum[warp] = eq;
-      sh.wsum2[warp] = gt;
-    }
-    __syncthreads();
-    uint32_t tie_before = 0, out_before = 0;
-    if constexpr (C > 1) {
-      if (threadIdx.x == 0) {
-        uint32_t g = 0, e = 0;
-        for (int w = 0; w < kWarps; ++w) {
-          g += sh.wsum2[w];
-          e += sh.wsum[w];
-        }
-        sh.xch[kXGt] = g;
-        sh.xch[kXEq] = e;
-      }
-      Cluster<C>::sync();
-      gather_xch<C>(sh);
-      for (unsigned q = 0; q < crank; ++q) {
-        const uint32_t room = krem > tie_before ? krem - tie_before : 0u;
-        out_before += sh.xall[q][kXGt] + min(sh.xall[q][kXEq], room);
-        tie_before += sh.xall[q][kXEq];
-      }
-    }
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      if (w < warp) {
-        const uint32_t room = krem > tie_before ? krem - tie_before : 0u;
-        out_before += sh.wsum2[w] + min(sh.wsum[w], room);
-        tie_before += sh.wsum[w];
-      }
-    }
-    const uint32_t lt = (1u << lane) - 1u;
-    for (uint32_t c0 = 0; c0 < cnt; c0 += 32) {
-      const uint32_t c = c0 + lane;
-      const uint32_t u = c < cnt ? rk[c] : 0u;
-      const bool is_gt = c < cnt && u > T;
-      const bool is_eq = c < cnt && u == T;
-      const uint32_t eqb = __ballot_sync(0xffffffffu, is_eq);
-      const bool take = is_gt || (is_eq && tie_before + __popc(eqb & lt) < krem);
-      const uint32_t tb = __ballot_sync(0xffffffffu, take);
-      if (take) {
-        const int j = rp[c];
-        const uint32_t slot = out_before + __popc(tb & lt);
-        out[slot] = j;
-        if (vout) vout[slot] = row[j];
-      }
-      out_before += __popc(tb);
-      tie_before += __popc(eqb);
-    }
-  }
-  // the next row (or, in a cluster, the other CTAs) may reuse shared memory
-  if constexpr (C > 1) Cluster<C>::sync();
-  else __syncthreads();
 }
 
 struct RowInfo {
@@ -751,7 +700,7 @@ __device__ __forceinline__ void prefetch_row(const float* row, int n) {
 // C == 1: a persistent grid; CTA b takes rows b, b + grid, ... and pulls its
 // next row into L2 at the start of each row.  C > 1: one row per cluster.
 template <int C, int CAP>
-__global__ void __launch_bounds__(kThreads, C == 1 ? (CAP <= 5120 ? 4 : 2) : 4)
+__global__ void __launch_bounds__(kThreads, C == 1 ? (CAP <= 5120 ? 4 : 2) : 2)
     topk_kernel(const float* __restrict__ logits, int64_t ld, const int32_t* __restrict__ cu_q,
                 const int32_t* __restrict__ cu_k, int B, int64_t total_q, int k,
                 int32_t* __restrict__ idx, float* __restrict__ val) {
@@ -781,7 +730,8 @@ __global__ void __launch_bounds__(kThreads, C == 1 ? (CAP <= 5120 ? 4 : 2) : 4)
 
 template <int C, int CAP>
 cudaError_t launch_t(const TopkArgs& a, cudaStream_t s) {
-  const size_t smem = sizeof(Shared<CAP>);
+  // clusters: rank 0 also holds the merge buffer (CAP keys, CAP positions)
+  const size_t smem = sizeof(Shared<CAP>) + (C > 1 ? 2 * CAP * sizeof(uint32_t) : 0);
   auto kern = topk_kernel<C, CAP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));

@@ -150,6 +150,48 @@ def test_topk_exact_adversarial_rows(k):
         assert np.array_equal(gi[q0:q1], o), f"sequence {b}"
 
 
+def test_topk_exact_few_long_rows():
+    # a batch of one-query sequences with a long cache (the shape that splits
+    # each row over several CTAs whose candidates are merged): random rows of
+    # many lengths around k, the no-threshold limit and the merge capacity;
+    # a rising row (all candidates in the last segment); a row with 8000
+    # evenly spread ties at the top (more candidates than one merged list
+    # holds); a row of two values
+    k = 2048
+    g = torch.Generator().manual_seed(808)
+    lens = [1, 2047, 2048, 2049, 4095, 4160, 4161, 5000, 5121, 9000, 16385, 30000, 65536,
+            70001, 131072]
+    rows = [torch.randn(n, generator=g) for n in lens]
+    lens.append(60000)
+    rows.append(torch.linspace(-1.0, 1.0, 60000))
+    lens.append(60000)
+    r = -torch.rand(60000, generator=g)
+    r[::7][:8000] = 1.0
+    rows.append(r)
+    lens.append(100000)
+    rows.append(torch.where(torch.rand(100000, generator=g) < 0.01, torch.tensor(2.0),
+                            torch.tensor(-2.0)))
+    B = len(rows)
+    ld = (max(lens) + 3) // 4 * 4
+    logits = torch.full((B, ld), float("nan"))
+    for i, rr in enumerate(rows):
+        logits[i, :lens[i]] = rr
+    cu_q = torch.arange(B + 1, dtype=torch.int32)
+    cu_k = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    idx = torch.full((B, k), -7, dtype=torch.int32, device="cuda")
+    val = torch.empty((B, k), dtype=torch.float32, device="cuda")
+    dsa.dsa_topk(logits.cuda(), cu_q.cuda(), cu_k.cuda(), B, 1, max(lens), k, idx, val,
+                 ld_logits=ld)
+    C.assert_no_device_error()
+    gi, gv = C.np_(idx), C.np_(val)
+    L = logits.numpy().astype(np.float64)
+    for b, n in enumerate(lens):
+        o = oracle.topk(L[b:b + 1, :n], 1, k)[0]
+        assert np.array_equal(gi[b], o), f"row {b} (n = {n})"
+        kept = o >= 0
+        assert np.array_equal(gv[b][kept], logits[b].numpy()[o[kept]]), f"values, row {b}"
+
+
 # --------------------------------------------------------------------------
 # Sparse attention (oracle fed the GPU's indices)
 # --------------------------------------------------------------------------
