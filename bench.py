@@ -73,6 +73,10 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kl", action="store_true")
     ap.add_argument("--no-mha", action="store_true")
+    ap.add_argument("--no-bwd", action="store_true")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="reference arm: query rows the oracle runs per step (default: one "
+                         "per host core, at least 8)")
     ap.add_argument("--split-sequence", action="store_true")
     ap.add_argument("--no-extra-configs", action="store_true",
                     help="measure only --config, not the other full-size configs")
@@ -308,6 +312,38 @@ def oracle_sample(wl, n_rows, seed):
     return dt, L / full_s, desc
 
 
+def oracle_sample_decode(wl, n_rows, seed):
+    """Runs the oracle on a sample of the rows of a one-query-per-sequence
+    batch (each row against its own cache) and extrapolates the time of the
+    whole batch with the per-row cost model.  The sample is stratified by
+    cache length: the shortest and the longest row and evenly spaced ranks
+    between (the seed is unused: the choice is deterministic)."""
+    import oracle
+    from tests import dsa_cases as C
+    lens = np.array([int(wl.cu_k[b + 1]) - int(wl.cu_k[b]) for b in range(wl.B)])
+    order = np.argsort(lens, kind="stable")
+    pick = sorted({int(i) for i in np.linspace(0, wl.B - 1, min(n_rows, wl.B)).round()})
+    rows = order[pick]
+    dt = 0.0
+    for b in rows:
+        q0, q1, k0, k1 = C.seq_slices(wl, int(b))
+        args = (C.np_(wl.q8[q0:q1]), C.np_(wl.q_scale[q0:q1]), C.np_(wl.w[q0:q1]),
+                C.np_(wl.k8[k0:k1]), C.np_(wl.k_scale[k0:k1]), C.bits(wl.q[q0:q1]),
+                C.bits(wl.kv[k0:k1]), np.array([k1 - k0 - 1], dtype=np.int64))
+        t0 = time.perf_counter()
+        oracle.forward_at(*args, wl.k, wl.scale)
+        dt += time.perf_counter() - t0
+    H_I, d_I, H = wl.q8.shape[1], wl.q8.shape[2], wl.q.shape[1]
+    full = float(oracle_row_cost(lens - 1, wl.k, H_I, d_I, H).sum())
+    part = float(oracle_row_cost(lens[rows] - 1, wl.k, H_I, d_I, H).sum())
+    full_s = dt * full / part
+    desc = (f"{len(rows)} of {wl.B} decode rows, stratified by cache length (shortest, longest "
+            f"and evenly spaced ranks); the whole batch's time extrapolated from the sample by "
+            f"the per-row flop model (n indexer pairs, min(n,k) attended pairs): "
+            f"{full_s:.1f} s")
+    return dt, wl.T_q / full_s, desc
+
+
 def oracle_threads():
     return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
 
@@ -493,6 +529,44 @@ def run_ours(args):
                     "traffic": ncu_traffic("attn_target_kernel", f"{cfg.name}")}
         del ws_kl, grad
 
+    # ---- the indexer's backward on the same workload (not part of the step):
+    # dq, dw, dk of a dense score-space gradient over every causal pair (the
+    # dense warm-up's case); the step's score buffer serves as that gradient
+    bwd_extra = None
+    if not args.no_bwd and world == 1 and len(st.parts) == 1 and H_I == 64 and d_I == 128:
+        dq = torch.empty((wl.T_q, H_I, d_I), dtype=torch.float32, device="cuda")
+        dw = torch.empty((wl.T_q, H_I), dtype=torch.float32, device="cuda")
+        dk = torch.empty((wl.T_k, d_I), dtype=torch.float32, device="cuda")
+
+        def bwd_call():
+            dsa.dsa_indexer_backward(wl.q8, wl.q_scale, wl.w, wl.k8, wl.k_scale, st.logits,
+                                     wl.cu_q, wl.cu_k, wl.B, wl.max_len_q, wl.max_len_k, dq, dw,
+                                     dk, ld_g=st.ld, stream=stream)
+        for _ in range(3):
+            bwd_call()
+        bev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(3)]
+        for e in bev:
+            flush.fill_(4.0)
+            e[0].record(stream)
+            bwd_call()
+            e[1].record(stream)
+        torch.cuda.synchronize()
+        if dsa.dsa_get_device_error() != 0:
+            raise RuntimeError("device error in the indexer backward measurement")
+        b_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in bev]))
+        # per causal pair: the FP8 gates twice (dq/dw pass and dk pass) and two
+        # bf16 gated sums, each 2*H_I*d_I flops; FP8 counted at half weight
+        # against the bf16 peak (it runs at twice the rate)
+        b_flops = c["causal_pairs"] * 2 * H_I * d_I * (1 + 2)
+        b_tf = b_flops / (b_ms / 1e3) / 1e12
+        bwd_extra = {"ms": round(b_ms, 4), "bound": "tensor", "achieved": round(b_tf, 2),
+                     "peak": bf16_peak, "unit": "TFLOP/s (bf16-equivalent)",
+                     "frac": round(b_tf / bf16_peak, 4),
+                     "work": "per causal pair: two FP8 gate products (half weight) and two "
+                             "bf16 gated sums, 2*H_I*d_I flops each",
+                     "traffic": None}
+        del dq, dw, dk
+
     # ---- the masked MHA short-prefill mode (not part of the step): dense
     # per-head attention over the selection, on its own short-prefill workload
     mha_extra = None
@@ -556,6 +630,7 @@ def run_ours(args):
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": st.launches() * args.steps, "clocks": clk,
         "indexer_kl": kl_extra,
+        "indexer_backward": bwd_extra,
         "masked_mha": mha_extra,
     }
     del st, wl
@@ -736,13 +811,18 @@ def run_reference(args):
         return
     cfg = W.CONFIGS[args.config]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    wl = W.make_prefill(args.config, device=dev)
-    n_rows = max(8, oracle_threads())
+    if cfg.decode:
+        wl = W.make_decode(args.config, device=dev)
+        sample = oracle_sample_decode
+    else:
+        wl = W.make_prefill(args.config, device=dev)
+        sample = oracle_sample
+    n_rows = args.rows if args.rows else max(8, oracle_threads())
     for i in range(args.warmup):
-        oracle_sample(wl, max(4, n_rows // 4), seed=1000 + i)
+        sample(wl, max(4, n_rows // 4), seed=1000 + i)
     secs, vals = [], []
     for i in range(args.steps):
-        dt, v, desc = oracle_sample(wl, n_rows, seed=i)
+        dt, v, desc = sample(wl, n_rows, seed=i)
         secs.append(dt)
         vals.append(v)
     step_s = float(np.mean(secs))
@@ -752,7 +832,9 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(step_s * 1e3, 1), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{cfg.name} (one causal prefill)", "L": cfg.L, "k": cfg.k,
+        "config": {"workload": f"{cfg.name} (" + ("one varlen decode batch" if cfg.decode else
+                                                  "one causal prefill") + ")",
+                   "L": cfg.L, "k": cfg.k,
                    "H": cfg.H, "H_I": cfg.H_I, "d_I": cfg.d_I,
                    "step": f"{n_rows} stratified query rows per step; value extrapolated to "
                            f"the whole workload by the per-row flop model"},
