@@ -74,6 +74,7 @@ def parse_args():
     ap.add_argument("--no-kl", action="store_true")
     ap.add_argument("--no-mha", action="store_true")
     ap.add_argument("--no-bwd", action="store_true")
+    ap.add_argument("--no-fused", action="store_true")
     ap.add_argument("--rows", type=int, default=0,
                     help="reference arm: query rows the oracle runs per step (default: one "
                          "per host core, at least 8)")
@@ -412,6 +413,54 @@ class Stepper:
         return c
 
 
+FUSED_CONFIGS = (2, 4)   # where the fused indexer + top-k is measured beside the step
+
+
+def measure_fused(dsa, st, steps, warmup, flush):
+    """The same step through dsa_forward_fused (indexer and top-k fused into
+    two passes over the keys; results equal the step's bit for bit), once per
+    chunk on the Stepper's buffers.  Returns (mean ms per step, launches per
+    step)."""
+    wl, s = st.wl, st.stream
+    d_I = wl.q8.shape[2]
+    need = max(dsa.dsa_forward_fused_workspace_size(p.T_q, p.T_k, p.B, p.max_len_k, p.k, d_I)
+               for _, p in st.parts)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+
+    def step():
+        for r0, p in st.parts:
+            r1 = r0 + p.T_q
+            dsa.dsa_forward_fused(p.q8, p.q_scale, p.w, p.k8, p.k_scale, p.q, p.kv, p.cu_q,
+                                  p.cu_k, p.B, p.max_len_q, p.max_len_k, p.k, p.scale,
+                                  st.out[r0:r1], st.lse[r0:r1], ws, idx_out=st.idx[r0:r1],
+                                  stream=s)
+    for _ in range(warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(float(i))
+        ev[i][0].record(s)
+        step()
+        ev[i][1].record(s)
+    torch.cuda.synchronize()
+    if dsa.dsa_get_device_error() != 0:
+        raise RuntimeError("device error in the fused measurement")
+    del ws
+    # per chunk: sample offsets, sample gather, three indexer launches (sampled,
+    # compact, recompute), threshold, candidate top-k, recompute top-k, attention
+    return float(np.mean([e[0].elapsed_time(e[1]) for e in ev])), 9 * len(st.parts)
+
+
+def fused_entry(ms, launches, unfused_ms):
+    return {"ms": round(ms, 4), "unfused_ms": round(unfused_ms, 4),
+            "speedup": round(unfused_ms / ms, 4), "gpu_launches_per_step": launches,
+            "what": "dsa_forward_fused: the indexer scores a 1/32 key sample for per-row "
+                    "thresholds, then appends only scores above them to candidate lists that "
+                    "top-k selects from; indices, outputs and lse equal the step's bit for bit"}
+
+
 def measure(dsa, st, steps, warmup, flush, clocks=None, barrier=None):
     """Warm-up, then `steps` timed steps with L2 flushed before each (outside
     the events).  Returns (mean ms per step, mean ms per stage [3], clocks)."""
@@ -633,6 +682,11 @@ def run_ours(args):
         "indexer_backward": bwd_extra,
         "masked_mha": mha_extra,
     }
+    if not args.no_fused and world == 1 and args.config in FUSED_CONFIGS:
+        f_steps = max(3, min(args.steps, 5))
+        f_ms, f_l = measure_fused(dsa, st, f_steps, 3, flush)
+        line["fused_indexer_topk"] = fused_entry(f_ms, f_l, step_ms)
+        line["gpu_launches"] += f_l * f_steps
     del st, wl
 
     # ---- the other full-size configurations at one GPU, each with its own
@@ -655,6 +709,10 @@ def run_ours(args):
                 "queries_per_step": xw.T_q, "chunks": xcfg.chunks,
                 "step_frac": round(xroof * 1e3 / xms, 4), "step_roof_ms": round(xroof * 1e3, 4),
                 "stages": xstages, "gpu_launches": xs.launches() * x_steps, "clocks": xclk}
+            if not args.no_fused and cid in FUSED_CONFIGS:
+                f_ms, f_l = measure_fused(dsa, xs, x_steps, 3, flush)
+                extra[xcfg.name]["fused_indexer_topk"] = fused_entry(f_ms, f_l, xms)
+                extra[xcfg.name]["gpu_launches"] += f_l * x_steps
             del xs, xw
         line["configs"] = extra
         line["gpu_launches"] += sum(v["gpu_launches"] for v in extra.values())

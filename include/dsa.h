@@ -163,6 +163,48 @@ DSA_API dsa_status_t dsa_forward(const void* q_fp8, const float* q_scale, const 
                          void* stream);
 
 /*
+ * Device workspace bytes for dsa_forward_fused (0 for unsupported sizes:
+ * k > 2048, max_len_k > 131072, d_I not 64 or 128).
+ */
+DSA_API size_t dsa_forward_fused_workspace_size(int64_t total_q, int64_t total_k, int B,
+                                                int max_len_k, int k, int d_I);
+
+/*
+ * dsa_forward with the indexer and the top-k fused into two passes over the
+ * keys, so the causal score matrix is not written to HBM and read back (blog,
+ * "What we would test": at long context the indexer's quadratic term is the
+ * cost that remains).  Same arguments, same results: idx, out and lse equal
+ * dsa_forward's bit for bit.
+ *
+ *  1. Every query is scored against a 1/32 sample of its sequence's keys
+ *     (positions 0, 32, 64, ...), and each row's threshold is the r0-th
+ *     largest score among the S samples it may see, r0 = E + 4 sqrt(E) + 8
+ *     with E = S k / (p + 1); rows of at most 4096 scores keep every score.
+ *  2. Every causal score is computed again (the same arithmetic as
+ *     dsa_indexer_logits) and only those at or above the row's threshold are
+ *     appended to the row's list of at most 5120 candidates.
+ *  3. A row with at least k candidates (and no more than the list holds) has
+ *     all of its k best scores in the list, ties included, and is selected
+ *     from it.  Any other row, and a row of massive ties, is recomputed on the
+ *     unfused path (dsa_indexer_logits and dsa_topk on those rows only).
+ *  4. dsa_sparse_mla_fwd on the indices.
+ *
+ *  workspace (device) dsa_forward_fused_workspace_size bytes, 16-byte aligned:
+ *           the sampled keys and their scores, thresholds, candidate lists,
+ *           and a full score matrix that only the recomputed rows touch.
+ *  Supported: as dsa_forward with H_I = 64, k <= 2048 and max_len_k <= 131072.
+ *  Errors: as dsa_forward; DSA_ERR_WORKSPACE for a missing or short workspace.
+ */
+DSA_API dsa_status_t dsa_forward_fused(const void* q_fp8, const float* q_scale, const float* w,
+                                       const void* k_fp8, const float* k_scale, const void* q,
+                                       const void* kv, const int32_t* cu_seqlens_q,
+                                       const int32_t* cu_seqlens_k, int B, int max_len_q,
+                                       int max_len_k, int64_t total_q, int64_t total_k, int H_I,
+                                       int d_I, int H, int d_qk, int d_v, int k, float sm_scale,
+                                       void* out, float* lse, int32_t* idx_out, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
+/*
  * dsa_forward for callers that cannot allocate device memory.  The pages have
  * no counterpart to this call; it exists for users of this library.
  *

@@ -17,7 +17,8 @@ __all__ = [
     "dsa_forward_workspace_size", "dsa_get_device_error", "dsa_forward_noalloc",
     "dsa_forward_host", "dsa_forward_host_workspace_size", "dsa_indexer_kl",
     "dsa_indexer_kl_workspace_size", "dsa_masked_mha_fwd", "dsa_masked_mha_workspace_size",
-    "dsa_debug_fault_injection", "dsa_indexer_backward", "EXPORTED",
+    "dsa_debug_fault_injection", "dsa_indexer_backward", "dsa_forward_fused",
+    "dsa_forward_fused_workspace_size", "EXPORTED",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -31,6 +32,7 @@ EXPORTED = (
     "dsa_forward_noalloc", "dsa_forward_host", "dsa_forward_host_workspace_size",
     "dsa_indexer_kl", "dsa_indexer_kl_workspace_size", "dsa_masked_mha_fwd",
     "dsa_masked_mha_workspace_size", "dsa_debug_fault_injection", "dsa_indexer_backward",
+    "dsa_forward_fused", "dsa_forward_fused_workspace_size",
 )
 
 STATUS = {
@@ -65,6 +67,9 @@ def load():
     lib.dsa_sparse_mla_fwd.argtypes = [P, P, P, P, P, I, I, I, I64, I64, I, I, I, I, F, P, P, P]
     lib.dsa_forward.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I64, I64, I, I, I, I, I, I, F,
                                 P, P, P, P, ctypes.c_size_t, P]
+    lib.dsa_forward_fused.argtypes = lib.dsa_forward.argtypes
+    lib.dsa_forward_fused_workspace_size.argtypes = [I64, I64, I, I, I, I]
+    lib.dsa_forward_fused_workspace_size.restype = ctypes.c_size_t
     lib.dsa_forward_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I64, I64, I, I, I, I,
                                         I, I, F, P, P, P, P]
     lib.dsa_forward_host.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I64, I64, I, I, I, I, I,
@@ -82,7 +87,7 @@ def load():
     lib.dsa_forward_host_workspace_size.argtypes = [I64, I, I, I, I, I, I, I, I]
     lib.dsa_forward_host_workspace_size.restype = ctypes.c_size_t
     for name in ("dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward",
-                 "dsa_forward_noalloc", "dsa_forward_host"):
+                 "dsa_forward_noalloc", "dsa_forward_host", "dsa_forward_fused"):
         getattr(lib, name).restype = I
     lib.dsa_forward_workspace_size.argtypes = [I64, I, I]
     lib.dsa_forward_workspace_size.restype = ctypes.c_size_t
@@ -260,6 +265,38 @@ def dsa_forward(q_fp8, q_scale, w, k_fp8, k_scale, q, kv, cu_seqlens_q, cu_seqle
                             _ptr(workspace), int(workspace.numel() * workspace.element_size()),
                             _stream(stream))
     _check(rc, "dsa_forward")
+
+
+def dsa_forward_fused_workspace_size(total_q, total_k, B, max_len_k, k, d_I) -> int:
+    return int(load().dsa_forward_fused_workspace_size(int(total_q), int(total_k), int(B),
+                                                       int(max_len_k), int(k), int(d_I)))
+
+
+def dsa_forward_fused(q_fp8, q_scale, w, k_fp8, k_scale, q, kv, cu_seqlens_q, cu_seqlens_k, B,
+                      max_len_q, max_len_k, k, sm_scale, out, lse, workspace, idx_out=None,
+                      stream=None):
+    """dsa_forward with the indexer and top-k fused into two passes over the
+    keys (the score matrix stays out of HBM); same results, bit for bit.  The
+    workspace holds dsa_forward_fused_workspace_size bytes."""
+    import torch
+    q8 = q_fp8.view(torch.uint8) if q_fp8.dtype == torch.float8_e4m3fn else q_fp8
+    k8 = k_fp8.view(torch.uint8) if k_fp8.dtype == torch.float8_e4m3fn else k_fp8
+    _need(q8, torch.uint8, "q_fp8", 3)
+    _need(k8, torch.uint8, "k_fp8", 2)
+    _need(q, torch.bfloat16, "q", 3)
+    _need(kv, torch.bfloat16, "kv", 2)
+    _need(out, torch.bfloat16, "out", 3)
+    _need(lse, torch.float32, "lse", 2)
+    _need(idx_out, torch.int32, "idx_out", 2)
+    T_q, H_I, d_I = q8.shape
+    _, H, d_qk = q.shape
+    rc = load().dsa_forward_fused(
+        _ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale), _ptr(q), _ptr(kv),
+        _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(B), int(max_len_q), int(max_len_k), int(T_q),
+        int(k8.shape[0]), int(H_I), int(d_I), int(H), int(d_qk), int(out.shape[2]), int(k),
+        float(sm_scale), _ptr(out), _ptr(lse), _ptr(idx_out), _ptr(workspace),
+        int(workspace.numel() * workspace.element_size()), _stream(stream))
+    _check(rc, "dsa_forward_fused")
 
 
 def dsa_forward_noalloc(q_fp8, q_scale, w, k_fp8, k_scale, q, kv, cu_seqlens_q, cu_seqlens_k, B,

@@ -465,6 +465,208 @@ dsa_status_t dsa_forward(const void* q_fp8, const float* q_scale, const float* w
                             total_q, total_k, H, d_qk, d_v, k, sm_scale, out, lse, stream);
 }
 
+namespace {
+
+// Regions of the fused forward's workspace, each 256-byte aligned.
+struct FusedLayout {
+  int64_t ld, ld_s, max_samples;
+  size_t logits, idx, k8_s, ks_s, cu_k_s, logits_s, thr, flags, cand_key, cand_pos, total;
+};
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+FusedLayout fused_layout(int64_t total_q, int64_t total_k, int B, int max_len_k, int k,
+                         int d_I) {
+  FusedLayout f;
+  f.ld = (static_cast<int64_t>(max_len_k) + 3) / 4 * 4;
+  const int64_t max_len_s = (static_cast<int64_t>(max_len_k) + dsa::kSampleStride - 1) /
+                            dsa::kSampleStride;
+  f.ld_s = (max_len_s + 3) / 4 * 4;
+  // sum over sequences of ceil(len_k / stride) <= total_k / stride + B
+  f.max_samples = total_k / dsa::kSampleStride + B;
+  size_t o = 0;
+  f.logits = o;   o += align256(static_cast<size_t>(total_q * f.ld) * 4);
+  f.idx = o;      o += align256(static_cast<size_t>(total_q) * k * 4);
+  f.k8_s = o;     o += align256(static_cast<size_t>(f.max_samples) * d_I);
+  f.ks_s = o;     o += align256(static_cast<size_t>(f.max_samples) * 4);
+  f.cu_k_s = o;   o += align256(static_cast<size_t>(B + 1) * 4);
+  f.logits_s = o; o += align256(static_cast<size_t>(total_q * f.ld_s) * 4);
+  f.thr = o;      o += align256(static_cast<size_t>(total_q) * 4);
+  f.flags = o;    o += align256(static_cast<size_t>(2 * total_q + 1) * 4);   // cnt, row_on, any
+  f.cand_key = o; o += align256(static_cast<size_t>(total_q) * dsa::kFusedCap * 4);
+  f.cand_pos = o; o += align256(static_cast<size_t>(total_q) * dsa::kFusedCap * 4);
+  f.total = o;
+  return f;
+}
+
+}  // namespace
+
+size_t dsa_forward_fused_workspace_size(int64_t total_q, int64_t total_k, int B, int max_len_k,
+                                        int k, int d_I) {
+  if (total_q < 0 || total_k < 0 || B < 0 || max_len_k < 0 || k < 1 || k > 2048 ||
+      max_len_k > dsa::kFusedMaxLenK || (d_I != 64 && d_I != 128))
+    return 0;
+  return fused_layout(total_q, total_k, B, max_len_k, k, d_I).total;
+}
+
+dsa_status_t dsa_forward_fused(const void* q_fp8, const float* q_scale, const float* w,
+                               const void* k_fp8, const float* k_scale, const void* q,
+                               const void* kv, const int32_t* cu_seqlens_q,
+                               const int32_t* cu_seqlens_k, int B, int max_len_q, int max_len_k,
+                               int64_t total_q, int64_t total_k, int H_I, int d_I, int H, int d_qk,
+                               int d_v, int k, float sm_scale, void* out, float* lse,
+                               int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  dsa_status_t st = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_len_q, max_len_k, total_q,
+                                 total_k);
+  if (st != DSA_OK) return st;
+  if (!q_fp8 || !q_scale || !w || !k_fp8 || !k_scale || !q || !kv || !out)
+    return DSA_ERR_INVALID_ARG;
+  if (!indexer_shape_ok(H_I, d_I) || H_I != 64) return DSA_ERR_UNSUPPORTED;
+  if (d_qk != 576 || d_v != 512 || !mla_heads_ok(H) || k < 1 || k > 2048 ||
+      max_len_k > dsa::kFusedMaxLenK)
+    return DSA_ERR_UNSUPPORTED;
+  if (!aligned16(q_fp8) || !aligned16(k_fp8) || (idx_out && !aligned16(idx_out)))
+    return DSA_ERR_ALIGNMENT;
+  if (total_q * H_I >= (int64_t(1) << 31) || total_k >= (int64_t(1) << 31) ||
+      total_q * static_cast<int64_t>(dsa::kFusedCap) >= (int64_t(1) << 40))
+    return DSA_ERR_UNSUPPORTED;
+  const FusedLayout f = fused_layout(total_q, total_k, B, max_len_k, k, d_I);
+  if (!workspace || workspace_bytes < f.total) return DSA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return DSA_ERR_ALIGNMENT;
+  if (total_q == 0 || B == 0) return DSA_OK;
+  if (total_k == 0) return DSA_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != DSA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* logits = reinterpret_cast<float*>(ws + f.logits);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + f.idx);
+  uint8_t* k8_s = ws + f.k8_s;
+  float* ks_s = reinterpret_cast<float*>(ws + f.ks_s);
+  int32_t* cu_k_s = reinterpret_cast<int32_t*>(ws + f.cu_k_s);
+  float* logits_s = reinterpret_cast<float*>(ws + f.logits_s);
+  float* thr = reinterpret_cast<float*>(ws + f.thr);
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(ws + f.flags);
+  uint32_t* row_on = cnt + total_q;
+  uint32_t* any_on = row_on + total_q;
+  uint32_t* cand_key = reinterpret_cast<uint32_t*>(ws + f.cand_key);
+  int32_t* cand_pos = reinterpret_cast<int32_t*>(ws + f.cand_pos);
+
+  if (cudaMemsetAsync(ws + f.flags, 0, static_cast<size_t>(2 * total_q + 1) * 4, s) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
+  // 1. the sampled keys and every query's scores against them
+  dsa::FusedSampleArgs sa;
+  sa.k8 = static_cast<const uint8_t*>(k_fp8);
+  sa.k_scale = k_scale;
+  sa.cu_k = cu_seqlens_k;
+  sa.B = B;
+  sa.d_I = d_I;
+  sa.max_samples = f.max_samples;
+  sa.k8_s = k8_s;
+  sa.k_scale_s = ks_s;
+  sa.cu_k_s = cu_k_s;
+  if ((st = from_cuda(dsa::launch_fused_sample(sa, s))) != DSA_OK) return st;
+  const CUtensorMapSwizzle swz =
+      d_I == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const int tile_n = (max_len_q <= 1 && H_I >= 16 && H_I <= 64) ? 64 : 256;
+  CUtensorMap tq, tk, tk_s;
+  if ((st = encode_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_fp8, total_q * H_I, d_I, 1,
+                      static_cast<uint32_t>(tile_n), d_I, swz)) != DSA_OK)
+    return st;
+  if ((st = encode_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, k_fp8, total_k, d_I, 1, 128, d_I,
+                      swz)) != DSA_OK)
+    return st;
+  if ((st = encode_2d(&tk_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, k8_s, f.max_samples, d_I, 1, 128,
+                      d_I, swz)) != DSA_OK)
+    return st;
+  dsa::IndexerArgs ia;
+  ia.q_scale = q_scale;
+  ia.w = w;
+  ia.k_scale = ks_s;
+  ia.cu_q = cu_seqlens_q;
+  ia.cu_k = cu_k_s;
+  ia.B = B;
+  ia.max_len_q = max_len_q;
+  ia.max_len_k = static_cast<int>((max_len_k + dsa::kSampleStride - 1) / dsa::kSampleStride);
+  ia.H_I = H_I;
+  ia.d_I = d_I;
+  ia.logits = logits_s;
+  ia.ld = f.ld_s;
+  ia.tile_n = tile_n;
+  ia.mode = dsa::kIdxRect;
+  if ((st = from_cuda(dsa::launch_indexer(tq, tk_s, ia, dev->num_sms, next_err(dev), s))) !=
+      DSA_OK)
+    return st;
+  dsa::FusedThresholdArgs ta;
+  ta.logits_s = logits_s;
+  ta.ld_s = f.ld_s;
+  ta.cu_q = cu_seqlens_q;
+  ta.cu_k = cu_seqlens_k;
+  ta.cu_k_s = cu_k_s;
+  ta.B = B;
+  ta.total_q = total_q;
+  ta.k = k;
+  ta.thr = thr;
+  if ((st = from_cuda(dsa::launch_fused_threshold(ta, s))) != DSA_OK) return st;
+  // 2. every causal score again, only those at or above the threshold kept
+  ia.k_scale = k_scale;
+  ia.cu_k = cu_seqlens_k;
+  ia.max_len_k = max_len_k;
+  ia.logits = logits;
+  ia.ld = f.ld;
+  ia.mode = dsa::kIdxCompact;
+  ia.thr = thr;
+  ia.cand_key = cand_key;
+  ia.cand_pos = cand_pos;
+  ia.cnt = cnt;
+  ia.cap = dsa::kFusedCap;
+  if ((st = from_cuda(dsa::launch_indexer(tq, tk, ia, dev->num_sms, next_err(dev), s))) !=
+      DSA_OK)
+    return st;
+  dsa::TopkCandArgs ca;
+  ca.cand_key = cand_key;
+  ca.cand_pos = cand_pos;
+  ca.cnt = cnt;
+  ca.cap = dsa::kFusedCap;
+  ca.cu_q = cu_seqlens_q;
+  ca.cu_k = cu_seqlens_k;
+  ca.B = B;
+  ca.max_len_k = max_len_k;
+  ca.total_q = total_q;
+  ca.k = k;
+  ca.idx = idx;
+  ca.row_on = row_on;
+  ca.any_on = any_on;
+  if ((st = from_cuda(dsa::launch_topk_candidates(ca, next_err(dev), s))) != DSA_OK) return st;
+  // 3. rows the candidate lists could not settle: the unfused path, on those
+  // rows only (both launches return at once when there are none)
+  ia.mode = dsa::kIdxCausal;
+  ia.row_on = row_on;
+  ia.any_on = any_on;
+  if ((st = from_cuda(dsa::launch_indexer(tq, tk, ia, dev->num_sms, next_err(dev), s))) !=
+      DSA_OK)
+    return st;
+  dsa::TopkArgs tka;
+  tka.logits = logits;
+  tka.ld = f.ld;
+  tka.cu_q = cu_seqlens_q;
+  tka.cu_k = cu_seqlens_k;
+  tka.B = B;
+  tka.max_len_q = max_len_q;
+  tka.max_len_k = max_len_k;
+  tka.total_q = total_q;
+  tka.k = k;
+  tka.idx = idx;
+  tka.val = nullptr;
+  tka.row_on = row_on;
+  tka.any_on = any_on;
+  if ((st = from_cuda(dsa::launch_topk(tka, next_err(dev), s))) != DSA_OK) return st;
+  return dsa_sparse_mla_fwd(q, kv, idx, cu_seqlens_q, cu_seqlens_k, B, max_len_q, max_len_k,
+                            total_q, total_k, H, d_qk, d_v, k, sm_scale, out, lse, stream);
+}
+
 void dsa_debug_fault_injection(uint64_t wait_limit_ns, int drop_first_key_load) {
   g_wait_limit_ns.store(wait_limit_ns);
   g_inject_indexer.store(drop_first_key_load ? dsa::kInjectDropFirstKeyLoad : 0u);

@@ -35,6 +35,7 @@
 #include <stdint.h>
 
 #include "internal.h"
+#include "keys.cuh"
 #include "ptx.cuh"
 
 namespace dsa {
@@ -60,6 +61,14 @@ struct Params {
   int n_kc;   // key chunks per sequence (virtual)
   int64_t n_items;
   int dense;  // 1: one query per sequence; items are the real (sequence, key chunk) pairs
+  int mode;   // kIdxCausal, kIdxRect or kIdxCompact
+  const float* thr;
+  uint32_t* cand_key;
+  int32_t* cand_pos;
+  uint32_t* cnt;
+  int cap;
+  const uint32_t* row_on;
+  const uint32_t* any_on;
   DevErr err;
 };
 
@@ -81,9 +90,12 @@ __device__ __forceinline__ bool fill_item(int b, int qg, int kc, int kb, const P
   it.len_q = cq1 - cq0;
   it.len_k = ck1 - ck0;
   it.q0 = qg * QPT;
-  if (it.q0 >= it.len_q || it.len_q > it.len_k) return false;
+  if (it.q0 >= it.len_q) return false;
+  if (P.mode != kIdxRect && it.len_q > it.len_k) return false;
   it.nq = min(QPT, it.len_q - it.q0);
-  const int p_max = it.len_k - it.len_q + it.q0 + it.nq - 1;
+  // the last key any query of the group reads (every key without the mask)
+  const int p_max =
+      P.mode == kIdxRect ? it.len_k - 1 : it.len_k - it.len_q + it.q0 + it.nq - 1;
   const int kbeg = kc * kb * kBlockK;
   const int kend = min(kbeg + kb * kBlockK, p_max + 1);
   if (kbeg >= kend) return false;
@@ -91,6 +103,12 @@ __device__ __forceinline__ bool fill_item(int b, int qg, int kc, int kb, const P
   it.nkb = (kend - kbeg + kBlockK - 1) / kBlockK;
   it.q_row0 = cq0 + it.q0;
   it.k_row0 = ck0;
+  if (P.row_on) {
+    // only groups holding a row to compute (every role reads the same flags)
+    bool any = false;
+    for (int i = 0; i < it.nq; ++i) any |= P.row_on[it.q_row0 + i] != 0u;
+    if (!any) return false;
+  }
   return true;
 }
 
@@ -153,13 +171,17 @@ struct Layout {
   static constexpr uint32_t kIdesc = instr_desc(kFmtE4M3, kFmtE4M3, 0, 0, kBlockK, kN);
 };
 
-template <int H_I, int D_I, int NT>
+// CMP: the read-out appends candidates (kIdxCompact) instead of storing scores.
+template <int H_I, int D_I, int NT, bool CMP>
 __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_k, const Params P) {
   using L = Layout<H_I, D_I, NT>;
   constexpr int kN = L::kN;
   constexpr int QPT = L::QPT;
+  // a launch on a row subset with no row set does nothing (the same word
+  // for every thread, read before any barrier or TMEM allocation)
+  if (P.any_on && *P.any_on == 0u) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -351,6 +373,11 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
     float* wq = wq_s + eg * kHalf;
     int64_t ac = 0;
     bool ok = true;
+    // compact mode: per query of this warpgroup, the last key it may append
+    // (its position or the sequence's last key) and its threshold
+    constexpr int QP = CMP ? QH : 1;
+    int lim_q[QP];
+    float thr_q[QP];
     for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
       Item it;
       if (!decode_item<QPT>(item, P, pre, it)) continue;
@@ -366,6 +393,14 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
           v = __ldg(P.w + o) * __ldg(P.q_scale + o);
         }
         wq[n] = v;
+      }
+      if constexpr (CMP) {
+#pragma unroll
+        for (int ql = 0; ql < QP; ++ql) {
+          const int qi = hf * QH + ql;
+          thr_q[ql] = qi < it.nq ? __ldg(P.thr + it.q_row0 + qi) : 0.f;
+          lim_q[ql] = qi < it.nq ? min(it.len_k - it.len_q + it.q0 + qi, it.len_k - 1) : -1;
+        }
       }
       named_bar_sync(bar_id, kEpiThreads);
       for (int j = 0; j < it.nkb; ++j, ++ac) {
@@ -422,15 +457,40 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
             }
           }
         }
-        if (s_local < it.len_k) {
-          const int p0 = it.len_k - it.len_q + it.q0;
+        const int p0 = it.len_k - it.len_q + it.q0;
+        if constexpr (CMP) {
+          // candidates: the causal scores at or above the row's threshold;
+          // one atomic per warp and query reserves their slots, lane order
+          // fills them
+#pragma unroll
+          for (int ql = 0; ql < QH; ++ql) {
+            float sum = 0.f;
+#pragma unroll
+            for (int ch = 0; ch < NCH; ++ch) sum += acc[ql][ch].x + acc[ql][ch].y;
+            const float sc = sum * ks;
+            const bool pass = s_local <= lim_q[ql] && sc >= thr_q[ql];
+            const uint32_t bal = __ballot_sync(0xffffffffu, pass);
+            if (bal != 0u) {
+              const int64_t r = it.q_row0 + hf * QH + ql;
+              uint32_t base = 0u;
+              if (lane == 0) base = atomicAdd(P.cnt + r, static_cast<uint32_t>(__popc(bal)));
+              base = __shfl_sync(0xffffffffu, base, 0);
+              const uint32_t slot = base + __popc(bal & ((1u << lane) - 1u));
+              if (pass && slot < static_cast<uint32_t>(P.cap)) {
+                const int64_t o = r * P.cap + slot;
+                P.cand_key[o] = order_key(sc);
+                P.cand_pos[o] = s_local;
+              }
+            }
+          }
+        } else if (s_local < it.len_k) {
 #pragma unroll
           for (int ql = 0; ql < QH; ++ql) {
             const int qi = hf * QH + ql;
             float sum = 0.f;
 #pragma unroll
             for (int ch = 0; ch < NCH; ++ch) sum += acc[ql][ch].x + acc[ql][ch].y;
-            if (qi < it.nq && s_local <= p0 + qi)
+            if (qi < it.nq && (P.mode == kIdxRect || s_local <= p0 + qi))
               st_global_stream(P.logits + static_cast<int64_t>(it.q_row0 + qi) * P.ld + s_local,
                                sum * ks);
           }
@@ -447,7 +507,7 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
   }
 }
 
-template <int H_I, int D_I, int NT>
+template <int H_I, int D_I, int NT, bool CMP>
 cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const IndexerArgs& a,
                      int num_sms, DevErr err, cudaStream_t s) {
   using L = Layout<H_I, D_I, NT>;
@@ -461,6 +521,14 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const Indexer
   P.ld = a.ld;
   P.B = a.B;
   P.dense = (L::QPT == 1 && a.max_len_q <= 1 && a.B <= kMaxDenseB) ? 1 : 0;
+  P.mode = a.mode;
+  P.thr = a.thr;
+  P.cand_key = a.cand_key;
+  P.cand_pos = a.cand_pos;
+  P.cnt = a.cnt;
+  P.cap = a.cap;
+  P.row_on = a.row_on;
+  P.any_on = a.any_on;
   P.n_qg = (a.max_len_q + L::QPT - 1) / L::QPT;
   P.n_kc = (a.max_len_k + kKbPerItem * kBlockK - 1) / (kKbPerItem * kBlockK);
   P.n_items = static_cast<int64_t>(a.B) * P.n_qg * P.n_kc;
@@ -480,7 +548,7 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const Indexer
   };
   while (gcd(P.n_kc, grid) != 1) ++P.n_kc;
   P.n_items = static_cast<int64_t>(a.B) * P.n_qg * P.n_kc;
-  auto kern = indexer_kernel<H_I, D_I, NT>;
+  auto kern = indexer_kernel<H_I, D_I, NT, CMP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(L::kSmem));
   if (e != cudaSuccess) return e;
@@ -492,10 +560,19 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const Indexer
 
 cudaError_t launch_indexer(const CUtensorMap& tq, const CUtensorMap& tk, const IndexerArgs& a,
                            int num_sms, DevErr err, cudaStream_t s) {
+  // the compact read-out is built for the 64-head indexer only
+  if (a.mode == kIdxCompact) {
+    if (a.H_I != 64) return cudaErrorInvalidValue;
+    if (a.d_I == 128 && a.tile_n == 256) return launch_t<64, 128, 256, true>(tq, tk, a, num_sms, err, s);
+    if (a.d_I == 128 && a.tile_n == 64) return launch_t<64, 128, 64, true>(tq, tk, a, num_sms, err, s);
+    if (a.d_I == 64 && a.tile_n == 256) return launch_t<64, 64, 256, true>(tq, tk, a, num_sms, err, s);
+    if (a.d_I == 64 && a.tile_n == 64) return launch_t<64, 64, 64, true>(tq, tk, a, num_sms, err, s);
+    return cudaErrorInvalidValue;
+  }
 #define DSA_IDX_CASE(h, d)                                                               \
-  if (a.H_I == h && a.d_I == d && a.tile_n == 256) return launch_t<h, d, 256>(tq, tk, a, num_sms, err, s);
+  if (a.H_I == h && a.d_I == d && a.tile_n == 256) return launch_t<h, d, 256, false>(tq, tk, a, num_sms, err, s);
 #define DSA_IDX_CASE_DECODE(h, d)                                                        \
-  if (a.H_I == h && a.d_I == d && a.tile_n == 64) return launch_t<h, d, 64>(tq, tk, a, num_sms, err, s);
+  if (a.H_I == h && a.d_I == d && a.tile_n == 64) return launch_t<h, d, 64, false>(tq, tk, a, num_sms, err, s);
   DSA_IDX_CASE(4, 64)
   DSA_IDX_CASE(8, 64)
   DSA_IDX_CASE(16, 64)

@@ -51,6 +51,7 @@
 #include <stdint.h>
 
 #include "internal.h"
+#include "keys.cuh"
 #include "ptx.cuh"
 
 namespace dsa {
@@ -66,18 +67,6 @@ constexpr int kBins = 2048;                // histogram bins (11 bits)
 constexpr int kBinBits = 11;
 constexpr int kBinsPerThread = kBins / kThreads;
 constexpr int kList = 512;                 // keys of the fine bin ranked directly
-
-__device__ __forceinline__ uint32_t order_key(float f) {
-  uint32_t u = __float_as_uint(f);
-  if (u == 0x80000000u) u = 0u;  // -0.0 -> +0.0
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// The float whose key is u (inverse of order_key on the keys it produces):
-// x >= key_float(order_key(y)) exactly when order_key(x) >= order_key(y).
-__device__ __forceinline__ float key_float(uint32_t u) {
-  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
-}
 
 // Bin shift that maps keys in [lo, hi] onto at most kBins bins.
 __device__ __forceinline__ int bin_shift(uint32_t lo, uint32_t hi) {
@@ -379,9 +368,11 @@ __device__ __forceinline__ uint32_t region_append(uint32_t* rk, int32_t* rp, uin
 // Steps 3 and 4 on one CTA: each warp holds `seg`, its contiguous share of
 // the row's m >= k candidates (the warps' shares in warp order give every
 // candidate once, in position order); (cmn, cmx) is this thread's part of the
-// candidates' key range.  Writes the k kept positions (and scores) to out.
+// candidates' key range.  Writes the k kept positions (and scores) to out and
+// returns true, or returns false without writing when too many keys share
+// the cut bin (massive ties), for the caller's exact fallback.
 template <int CAP>
-__device__ void select_and_output(const float* __restrict__ row, int n, int k,
+__device__ bool select_and_output(const float* __restrict__ row, int n, int k,
                                   int32_t* __restrict__ out, float* __restrict__ vout,
                                   Shared<CAP>& sh, const Seg seg, uint32_t cmn, uint32_t cmx) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -422,11 +413,7 @@ __device__ void select_and_output(const float* __restrict__ row, int n, int k,
     });
     __syncthreads();
     const uint32_t total = sh.list_n;
-    if (total > static_cast<uint32_t>(kList)) {
-      // too many keys share the cut bin (massive ties): exact fallback
-      topk_row_global(row, n, k, out, vout, sh);
-      return;
-    }
+    if (total > static_cast<uint32_t>(kList)) return false;   // (uniform: sh.list_n)
     // rank every key of the bin against all of them: the kk-th largest is the
     // key with fewer than kk keys above it and at least kk at or above it
     if (threadIdx.x == 0) sh.res_key = 0u;
@@ -491,6 +478,7 @@ __device__ void select_and_output(const float* __restrict__ row, int n, int k,
     tie_before += __popc(eqb);
   }
   __syncthreads();   // the next row may reuse shared memory
+  return true;
 }
 
 // One row, by every thread of every CTA of the cluster (C > 1: the merged
@@ -617,7 +605,8 @@ __device__ void topk_row(const float* __restrict__ row, int n, int k, int32_t* _
       topk_row_global(row, n, k, out, vout, sh);
       return;
     }
-    select_and_output<CAP>(row, n, k, out, vout, sh, Seg{rk, rp, sh.wcnt[warp]}, cmn, cmx);
+    if (!select_and_output<CAP>(row, n, k, out, vout, sh, Seg{rk, rp, sh.wcnt[warp]}, cmn, cmx))
+      topk_row_global(row, n, k, out, vout, sh);
   } else {
     // merge: every CTA stores its regions, in warp order, into rank 0's merge
     // buffer after those of the lower ranks
@@ -664,7 +653,9 @@ __device__ void topk_row(const float* __restrict__ row, int n, int k, int32_t* _
       cmn = min(cmn, mk[c]);
       cmx = max(cmx, mk[c]);
     }
-    select_and_output<CAP>(row, n, k, out, vout, sh, Seg{mk + s0, mp + s0, s1 - s0}, cmn, cmx);
+    if (!select_and_output<CAP>(row, n, k, out, vout, sh, Seg{mk + s0, mp + s0, s1 - s0}, cmn,
+                                cmx))
+      topk_row_global(row, n, k, out, vout, sh);
   }
 }
 
@@ -703,16 +694,22 @@ template <int C, int CAP>
 __global__ void __launch_bounds__(kThreads, C == 1 ? (CAP <= 5120 ? 4 : 2) : 2)
     topk_kernel(const float* __restrict__ logits, int64_t ld, const int32_t* __restrict__ cu_q,
                 const int32_t* __restrict__ cu_k, int B, int64_t total_q, int k,
-                int32_t* __restrict__ idx, float* __restrict__ val) {
+                int32_t* __restrict__ idx, float* __restrict__ val,
+                const uint32_t* __restrict__ row_on, const uint32_t* __restrict__ any_on) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   Shared<CAP>& sh = *reinterpret_cast<Shared<CAP>*>(smem_raw);
+  // a launch on a row subset with no row set does nothing
+  if (any_on && *any_on == 0u) return;
+  auto on = [&](int64_t r) { return row_on == nullptr || row_on[r] != 0u; };
   if constexpr (C == 1) {
     int64_t r = blockIdx.x;
+    while (r < total_q && !on(r)) r += gridDim.x;
     if (r >= total_q) return;
     RowInfo cur = row_info(r, logits, ld, cu_q, cu_k, B);
     if (threadIdx.x == 0) prefetch_row(cur.row, cur.n);
-    for (; r < total_q; r += gridDim.x) {
-      const int64_t rn = r + gridDim.x;
+    while (r < total_q) {
+      int64_t rn = r + gridDim.x;
+      while (rn < total_q && !on(rn)) rn += gridDim.x;
       RowInfo nxt = cur;
       if (rn < total_q) {
         nxt = row_info(rn, logits, ld, cu_q, cu_k, B);
@@ -720,9 +717,11 @@ __global__ void __launch_bounds__(kThreads, C == 1 ? (CAP <= 5120 ? 4 : 2) : 2)
       }
       topk_row<1, CAP>(cur.row, cur.n, k, idx + r * k, val ? val + r * k : nullptr, sh);
       cur = nxt;
+      r = rn;
     }
   } else {
     const int64_t r = blockIdx.x / C;
+    if (!on(r)) return;   // (the whole cluster alike)
     const RowInfo ri = row_info(r, logits, ld, cu_q, cu_k, B);
     topk_row<C, CAP>(ri.row, ri.n, k, idx + r * k, val ? val + r * k : nullptr, sh);
   }
@@ -760,9 +759,91 @@ cudaError_t launch_t(const TopkArgs& a, cudaStream_t s) {
   cfg.attrs = attr;
   cfg.numAttrs = C > 1 ? 1 : 0;
   e = cudaLaunchKernelEx(&cfg, kern, a.logits, a.ld, a.cu_q, a.cu_k, a.B, a.total_q, a.k, a.idx,
-                         a.val);
+                         a.val, a.row_on, a.any_on);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+// Top-k of rows whose candidates an indexer launch in compact mode listed
+// (every causal score at or above the row's threshold, in no particular
+// order).  With m >= k candidates the row's k best scores are all among them,
+// ties included, so the selection equals the one over the whole row.  The
+// candidates are put in position order through a bitmap of their positions
+// (a prefix over its words ranks each one), then selected as above.  A row
+// with fewer than k candidates, more than the list holds, or too many keys in
+// the cut bin is marked in row_on (and any_on set) for the unfused path.
+template <int CAP>
+__global__ void __launch_bounds__(kThreads, 2)
+    topk_cand_kernel(const uint32_t* __restrict__ cand_key, const int32_t* __restrict__ cand_pos,
+                     const uint32_t* __restrict__ cnt, int cap, const int32_t* __restrict__ cu_q,
+                     const int32_t* __restrict__ cu_k, int B, int64_t total_q, int k,
+                     int32_t* __restrict__ idx, uint32_t* __restrict__ row_on,
+                     uint32_t* __restrict__ any_on, int max_words) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  Shared<CAP>& sh = *reinterpret_cast<Shared<CAP>*>(smem_raw);
+  uint32_t* bm = reinterpret_cast<uint32_t*>(&sh + 1);        // position bitmap
+  uint16_t* wpre = reinterpret_cast<uint16_t*>(bm + max_words);  // candidates before each word
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int64_t r = blockIdx.x; r < total_q; r += gridDim.x) {
+    const int n = row_info(r, nullptr, 0, cu_q, cu_k, B).n;
+    int32_t* out = idx + r * k;
+    if (n <= k) {
+      for (int j = threadIdx.x; j < k; j += kThreads) out[j] = j < n ? j : -1;
+      continue;
+    }
+    const uint32_t m = cnt[r];
+    if (m < static_cast<uint32_t>(k) || m > static_cast<uint32_t>(CAP) ||
+        m > static_cast<uint32_t>(cap)) {
+      if (threadIdx.x == 0) {
+        row_on[r] = 1u;
+        *any_on = 1u;
+      }
+      continue;
+    }
+    const uint32_t* ck = cand_key + r * cap;
+    const int32_t* cp = cand_pos + r * cap;
+    const int words = (n + 31) >> 5;
+    for (int w = threadIdx.x; w < words; w += kThreads) bm[w] = 0u;
+    __syncthreads();
+    for (uint32_t i = threadIdx.x; i < m; i += kThreads) {
+      const int pos = cp[i];
+      atomicOr(bm + (pos >> 5), 1u << (pos & 31));
+    }
+    __syncthreads();
+    const int wpt = (words + kThreads - 1) / kThreads;
+    const int w0 = min(static_cast<int>(threadIdx.x) * wpt, words), w1 = min(w0 + wpt, words);
+    uint32_t run = 0;
+    for (int w = w0; w < w1; ++w) run += __popc(bm[w]);
+    uint32_t tot;
+    run = block_excl_scan(run, sh, &tot);
+    for (int w = w0; w < w1; ++w) {
+      wpre[w] = static_cast<uint16_t>(run);
+      run += __popc(bm[w]);
+    }
+    __syncthreads();
+    for (uint32_t i = threadIdx.x; i < m; i += kThreads) {
+      const int pos = cp[i];
+      const uint32_t rank = wpre[pos >> 5] + __popc(bm[pos >> 5] & ((1u << (pos & 31)) - 1u));
+      sh.cand_key[rank] = ck[i];
+      sh.cand_pos[rank] = pos;
+    }
+    __syncthreads();
+    const uint32_t share = (m + kWarps - 1) / kWarps;
+    const uint32_t s0 = min(warp * share, m), s1 = min(s0 + share, m);
+    uint32_t cmn = 0xffffffffu, cmx = 0u;
+    for (uint32_t c = s0 + lane; c < s1; c += 32) {
+      cmn = min(cmn, sh.cand_key[c]);
+      cmx = max(cmx, sh.cand_key[c]);
+    }
+    if (!select_and_output<CAP>(nullptr, n, k, out, nullptr, sh,
+                                Seg{sh.cand_key + s0, sh.cand_pos + s0, s1 - s0}, cmn, cmx)) {
+      if (threadIdx.x == 0) {
+        row_on[r] = 1u;
+        *any_on = 1u;
+      }
+      __syncthreads();
+    }
+  }
 }
 
 }  // namespace
@@ -776,6 +857,32 @@ cudaError_t launch_topk(const TopkArgs& a, DevErr err, cudaStream_t s) {
   if (split) return launch_t<kSplitC, 5120>(a, s);
   if (a.k <= 2048) return launch_t<1, 5120>(a, s);
   return launch_t<1, 8192>(a, s);
+}
+
+cudaError_t launch_topk_candidates(const TopkCandArgs& a, DevErr err, cudaStream_t s) {
+  (void)err;
+  if (a.total_q == 0) return cudaSuccess;
+  if (a.k > 2048 || a.max_len_k > kFusedMaxLenK || a.cap > kFusedCap) return cudaErrorInvalidValue;
+  constexpr int CAP = kFusedCap;
+  const int max_words = (a.max_len_k + 31) / 32;
+  const size_t smem = sizeof(Shared<CAP>) + static_cast<size_t>(max_words) * 4 +
+                      (static_cast<size_t>(max_words) * 2 + 15) / 16 * 16;
+  auto kern = topk_cand_kernel<CAP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148, per_sm = 1;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) !=
+          cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  int64_t grid = a.total_q;
+  if (grid > static_cast<int64_t>(sms) * per_sm) grid = static_cast<int64_t>(sms) * per_sm;
+  kern<<<static_cast<unsigned>(grid), kThreads, smem, s>>>(
+      a.cand_key, a.cand_pos, a.cnt, a.cap, a.cu_q, a.cu_k, a.B, a.total_q, a.k, a.idx, a.row_on,
+      a.any_on, max_words);
+  return cudaGetLastError();
 }
 
 }  // namespace dsa

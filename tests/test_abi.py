@@ -197,3 +197,27 @@ def test_masked_mha_checks_before_any_device_call():
     assert call(ws=None) == WORKSPACE
     assert call(nbytes=need - 1) == WORKSPACE
     assert call(q=_fake(0x10008)) == ALIGN
+
+
+def test_forward_fused_checks_before_any_device_call():
+    lib = dsa.load()
+    p = _fake()
+    T, Tk, B, L, k, d_I = 64, 64, 1, 64, 32, 128
+    need = dsa.dsa_forward_fused_workspace_size(T, Tk, B, L, k, d_I)
+    assert need > dsa.dsa_forward_workspace_size(T, L, k)
+    # sizes it does not support
+    assert dsa.dsa_forward_fused_workspace_size(T, Tk, B, L, 4096, d_I) == 0
+    assert dsa.dsa_forward_fused_workspace_size(T, Tk, B, 131073, k, d_I) == 0
+    assert dsa.dsa_forward_fused_workspace_size(T, Tk, B, L, k, 96) == 0
+
+    def call(ws=p, nbytes=need, k=k, H_I=64, mlk=L):
+        return lib.dsa_forward_fused(p, p, p, p, p, p, p, p, p, B, L, mlk, T, Tk, H_I, d_I, 128,
+                                     576, 512, k, 0.05, p, p, None, ws, nbytes, None)
+    assert call(ws=None) == WORKSPACE
+    assert call(nbytes=need - 1) == WORKSPACE
+    assert call(ws=_fake(0x10008)) == ALIGN
+    assert call(k=4096) == UNSUPPORTED               # the candidate lists hold 5120 entries
+    assert call(H_I=48) == UNSUPPORTED
+    assert call(H_I=32) == UNSUPPORTED               # the compact read-out is 64-head only
+    if not _have_gpu():
+        assert call() == CUDA                        # no device: fails loudly
