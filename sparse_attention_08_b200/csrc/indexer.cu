@@ -262,6 +262,8 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int64_t qc = 0, kc = 0;
+      int st = 0;            // key stage of tile kc and its fill parity
+      uint32_t kpar = 0u;
       bool ok = true;
       const bool dropped = (P.err.inject & kInjectDropFirstKeyLoad) != 0;
       // the key tiles are read by every query group: keep them in L2 while
@@ -276,9 +278,7 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
         tma_load_2d(sbase + L::kOffQ + qb * L::kQBytes, &tmap_q, 0, it.q_row0 * H_I, q_full(qb));
         ++qc;
         for (int j = 0; j < it.nkb; ++j) {
-          const int st = static_cast<int>(kc % kStages);
-          const uint32_t par = static_cast<uint32_t>(((kc / kStages) & 1) ^ 1);
-          if (!(ok = mbar_wait(k_empty(st), par, P.err))) break;
+          if (!(ok = mbar_wait(k_empty(st), kpar ^ 1u, P.err))) break;
           // test hook: the first key tile is never loaded, so the MMA
           // issuer's bounded wait for it runs out
           if (kc != 0 || !dropped) {
@@ -287,6 +287,10 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
                              it.k_row0 + (it.kb0 + j) * kBlockK, k_full(st), keep);
           }
           ++kc;
+          if (++st == kStages) {
+            st = 0;
+            kpar ^= 1u;
+          }
         }
       }
       if (!ok) *abort_flag = 1;
@@ -309,7 +313,12 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
     // a tile's MMAs; every operand is warp-uniform and the descriptors are
     // built once: a stage or query buffer adds a multiple of its size (in
     // 16-byte units) to the start-address field.
-    int64_t qc = 0, kc = 0, ac = 0;
+    // ring positions as running counters (the warp shares its scheduler
+    // with the read-out warps, so every instruction per tile counts):
+    // key stage st and its fill parity, accumulator buffer ab and its phase
+    int64_t qc = 0;
+    int st = 0, ab = 0;
+    uint32_t kpar = 0u, apar = 0u;
     bool ok = true;
     const uint64_t a0 = smem_desc(sbase + L::kOffK, 16, L::kSbo, L::kSwizzle);
     const uint64_t b0 = smem_desc(sbase + L::kOffQ, 16, L::kSbo, L::kSwizzle);
@@ -320,10 +329,7 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
       if (!(ok = warp_wait(q_full(qb), static_cast<uint32_t>((qc >> 1) & 1), P.err))) break;
       const uint64_t bq = b0 + ((static_cast<uint32_t>(qb) * L::kQBytes) >> 4);
       for (int j = 0; j < it.nkb; ++j) {
-        const int st = static_cast<int>(kc % kStages);
-        const int ab = static_cast<int>(ac % kBufs);
-        ok = warp_wait(k_full(st), static_cast<uint32_t>((kc / kStages) & 1), P.err) &&
-             warp_wait(acc_empty(ab), static_cast<uint32_t>(((ac / kBufs) & 1) ^ 1), P.err);
+        ok = warp_wait(k_full(st), kpar, P.err) && warp_wait(acc_empty(ab), apar ^ 1u, P.err);
         if (!ok) break;
         tc_fence_after();
         const uint64_t ak = a0 + ((static_cast<uint32_t>(st) * L::kKBytes) >> 4);
@@ -336,8 +342,14 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
           mma_commit(acc_full(ab));
         }
         __syncwarp();
-        ++kc;
-        ++ac;
+        if (++st == kStages) {
+          st = 0;
+          kpar ^= 1u;
+        }
+        if (++ab == kBufs) {
+          ab = 0;
+          apar ^= 1u;
+        }
       }
       if (!ok) break;
       if (elect_one()) mma_commit(q_empty(qb));
