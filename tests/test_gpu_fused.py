@@ -94,3 +94,12 @@ def test_fused_equals_unfused_config4_chunks():
     for c in (0, 3, 7):
         _same_as_unfused(W.chunk_of(full, c, C_))
         torch.cuda.empty_cache()
+
+
+def test_fused_equals_unfused_config2_bench_size():
+    # the L = 32768 prefill, the size the bench measures the fused path at
+    _same_as_unfused(W.make_prefill(2, device="cuda"))
+
+
+def test_fused_equals_unfused_config3_all_rows():
+    _same_as_unfused(W.make_decode(3, device="cuda"))
