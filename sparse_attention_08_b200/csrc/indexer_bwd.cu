@@ -54,6 +54,21 @@ __device__ __forceinline__ float e4m3_value(uint32_t b) {
   return (b & 0x80u) ? -v : v;
 }
 
+// Two e4m3 codes (bits 0-7 and 8-15 of two) -> bf16x2 (first in the low
+// half), exactly: the hardware widens e4m3 to f16 (which holds every e4m3
+// value), and f16 -> f32 -> bf16 loses nothing for these values either.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+      : "=r"(h2)
+      : "r"(two));
+  float lo, hi;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(h2));
+  return pack_bf16x2(lo, hi);
+}
+
 // ---------------------------------------------------------------------------
 // dq, dw
 // ---------------------------------------------------------------------------
@@ -263,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 4; ++e) {
             const uint32_t wv = wd[2 * hh + (e >> 1)];
             const int sh = 16 * (e & 1);
-            pk[e] = pack_bf16x2(e4m3_value((wv >> sh) & 0xFFu), e4m3_value((wv >> (sh + 8)) & 0xFFu));
+            pk[e] = e4m3x2_to_bf16x2((wv >> sh) & 0xFFFFu);
           }
           const int d0 = 16 * c16 + 8 * hh;             // first dim of this 8-dim piece
           *reinterpret_cast<uint4*>(hrow + (d0 / 64) * kAtom + ((((d0 % 64) / 8) ^ (s & 7)) << 4)) =
@@ -539,8 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < 4; ++e) {
               const uint32_t wv = wd[2 * hh + (e >> 1)];
               const int sh = 16 * (e & 1);
-              pk[e] = pack_bf16x2(e4m3_value((wv >> sh) & 0xFFu),
-                                  e4m3_value((wv >> (sh + 8)) & 0xFFu));
+              pk[e] = e4m3x2_to_bf16x2((wv >> sh) & 0xFFFFu);
             }
             const int d0 = 16 * c16 + 8 * hh;
             *reinterpret_cast<uint4*>(dst + (d0 / 64) * kBAtom +
