@@ -31,6 +31,15 @@
 // queries); warp w reads TMEM lanes 32*(w%4)...  The ReLU / weighted-sum
 // read-out costs about as many issue slots as the MMA takes cycles, so it
 // is spread over four warps per sub-partition to hide TMEM and FMA latency.
+//
+// Read-out modes (the fused indexer + top-k, fused.cu): kIdxRect stores the
+// score of every key of the sequence (no causal mask; for the sampled keys),
+// and kIdxCompact (a separate instantiation, 64 heads) stores no scores but
+// appends the (order key, position) of each causal score at or above its
+// row's threshold to the row's candidate list: one ballot per warp and
+// query, one atomic on the row's count to reserve the slots.  A launch may be
+// limited to the query groups that hold a flagged row (row_on), and does
+// nothing while no row is flagged (any_on).
 #include <cuda_runtime.h>
 #include <stdint.h>
 

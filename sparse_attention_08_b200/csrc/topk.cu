@@ -45,6 +45,12 @@
 // ordered ballot-scan compaction.  Both routes give the same, unique answer.
 // Every decision that changes how many cluster barriers a CTA passes is taken
 // from values that all CTAs of the cluster read alike.
+//
+// The fused indexer + top-k (fused.cu) hands this file candidate lists
+// instead of score rows: topk_cand_kernel puts a row's candidates in position
+// order through a bitmap of their positions and runs steps 3 and 4 on them;
+// a row it cannot settle is flagged, and topk_kernel then runs on the flagged
+// rows only (row_on).
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <math.h>
