@@ -318,53 +318,52 @@ __global__ void __launch_bounds__(Layout<H_I, D_I, NT>::kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // The whole warp walks the items in lockstep and one elected lane issues
-    // a tile's MMAs; every operand is warp-uniform and the descriptors are
-    // built once: a stage or query buffer adds a multiple of its size (in
-    // 16-byte units) to the start-address field.
-    // ring positions as running counters (the warp shares its scheduler
-    // with the read-out warps, so every instruction per tile counts):
-    // key stage st and its fill parity, accumulator buffer ab and its phase
-    int64_t qc = 0;
-    int st = 0, ab = 0;
-    uint32_t kpar = 0u, apar = 0u;
+    // Lane 0 alone walks the items, waits and issues a tile's MMAs: the warp
+    // shares its scheduler with the read-out warps, so every instruction per
+    // tile counts (no broadcast of wait verdicts, no elect, no warp sync).
+    // The descriptors are built once (a stage or query buffer adds a multiple
+    // of its size, in 16-byte units, to the start-address field) and the ring
+    // positions are running counters: key stage st and its fill parity,
+    // accumulator buffer ab and its phase.
     bool ok = true;
-    const uint64_t a0 = smem_desc(sbase + L::kOffK, 16, L::kSbo, L::kSwizzle);
-    const uint64_t b0 = smem_desc(sbase + L::kOffQ, 16, L::kSbo, L::kSwizzle);
-    for (int64_t item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
-      Item it;
-      if (!decode_item<QPT>(item, P, pre, it)) continue;
-      const int qb = static_cast<int>(qc & 1);
-      if (!(ok = warp_wait(q_full(qb), static_cast<uint32_t>((qc >> 1) & 1), P.err))) break;
-      const uint64_t bq = b0 + ((static_cast<uint32_t>(qb) * L::kQBytes) >> 4);
-      for (int j = 0; j < it.nkb; ++j) {
-        ok = warp_wait(k_full(st), kpar, P.err) && warp_wait(acc_empty(ab), apar ^ 1u, P.err);
-        if (!ok) break;
-        tc_fence_after();
-        const uint64_t ak = a0 + ((static_cast<uint32_t>(st) * L::kKBytes) >> 4);
-        const uint32_t d = tmem + static_cast<uint32_t>(ab) * kN;
-        if (elect_one()) {
+    if (lane == 0) {
+      int64_t qc = 0;
+      int st = 0, ab = 0;
+      uint32_t kpar = 0u, apar = 0u;
+      const uint64_t a0 = smem_desc(sbase + L::kOffK, 16, L::kSbo, L::kSwizzle);
+      const uint64_t b0 = smem_desc(sbase + L::kOffQ, 16, L::kSbo, L::kSwizzle);
+      for (int64_t item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+        Item it;
+        if (!decode_item<QPT>(item, P, pre, it)) continue;
+        const int qb = static_cast<int>(qc & 1);
+        if (!(ok = mbar_wait(q_full(qb), static_cast<uint32_t>((qc >> 1) & 1), P.err))) break;
+        const uint64_t bq = b0 + ((static_cast<uint32_t>(qb) * L::kQBytes) >> 4);
+        for (int j = 0; j < it.nkb; ++j) {
+          ok = mbar_wait(k_full(st), kpar, P.err) && mbar_wait(acc_empty(ab), apar ^ 1u, P.err);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t ak = a0 + ((static_cast<uint32_t>(st) * L::kKBytes) >> 4);
+          const uint32_t d = tmem + static_cast<uint32_t>(ab) * kN;
 #pragma unroll
           for (int kk = 0; kk < D_I / 32; ++kk)
             mma_f8(d, ak + (kk * 32 >> 4), bq + (kk * 32 >> 4), L::kIdesc, kk > 0 ? 1u : 0u);
           mma_commit(k_empty(st));
           mma_commit(acc_full(ab));
+          if (++st == kStages) {
+            st = 0;
+            kpar ^= 1u;
+          }
+          if (++ab == kBufs) {
+            ab = 0;
+            apar ^= 1u;
+          }
         }
-        __syncwarp();
-        if (++st == kStages) {
-          st = 0;
-          kpar ^= 1u;
-        }
-        if (++ab == kBufs) {
-          ab = 0;
-          apar ^= 1u;
-        }
+        if (!ok) break;
+        mma_commit(q_empty(qb));
+        ++qc;
       }
-      if (!ok) break;
-      if (elect_one()) mma_commit(q_empty(qb));
-      __syncwarp();
-      ++qc;
     }
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     // every MMA issued by this warp completes before TMEM is released
     mma_commit_warp(drain_bar);
     if (lane == 0) {
